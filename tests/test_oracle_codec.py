@@ -1,0 +1,248 @@
+"""Pins of the oracle's quantize / dequantize / KV codec (no GPU).
+
+Each check ties the oracle to something other than itself: numpy binary32
+arithmetic plus ml_dtypes / torch format conversions for the recipe's steps,
+exact round trips of tensors built from representable values, the per-block
+error bound of the format, the size ratio printed on the pages, and algebraic
+invariants of the KV codec.
+"""
+import json
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_w4a4_quantized_08_b200 import workloads as wl
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "page_facts.json")
+F32 = np.float32
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def unpack(codes: np.ndarray) -> np.ndarray:
+    lo = codes & 0xF
+    hi = codes >> 4
+    return np.stack([lo, hi], axis=-1).reshape(codes.shape[0], -1)
+
+
+# ------------------------------------------------------------------ recipe pins
+def _independent_quantize(x32: np.ndarray):
+    """The recipe's steps in numpy binary32 + ml_dtypes conversions."""
+    amax = np.max(np.abs(x32))
+    s_t = F32(amax) / F32(2688.0)
+    rows, cols = x32.shape
+    blocks = x32.reshape(rows, cols // 16, 16)
+    amax_b = np.max(np.abs(blocks), axis=2).astype(F32)
+    if s_t == 0:
+        sb = np.zeros_like(amax_b, dtype=np.uint8)
+    else:
+        r = amax_b / (F32(6.0) * s_t)
+        sb = np.minimum(r, F32(448.0)).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    sbv = sb.view(ml_dtypes.float8_e4m3fn).astype(F32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        d = (sbv * s_t)[:, :, None]
+        y = blocks / d
+    q = np.clip(y, -6, 6).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    q[np.broadcast_to((sb == 0)[:, :, None], q.shape)] = 0
+    return q.reshape(rows, cols), sb, s_t
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_quantize_matches_numpy_steps(orc, dtype):
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(64, 256, generator=g)
+    x[3, 17] = 40.0  # outlier
+    x[7, 32:48] = 0.0  # an all-zero block
+    x[9, 0:16] *= 1e-4  # a block whose scale is subnormal in E4M3
+    xn = x.numpy()
+    if dtype == "bf16":
+        bits = bf16_bits(xn)
+        x32 = bits_to_f32(bits)
+        codes, sf, st = orc.quantize(bits)
+    else:
+        x32 = xn.astype(F32)
+        codes, sf, st = orc.quantize(x32)
+    q_ref, sb_ref, st_ref = _independent_quantize(x32)
+    assert st == st_ref
+    np.testing.assert_array_equal(sf, sb_ref)
+    np.testing.assert_array_equal(unpack(codes), q_ref)
+    assert np.all(sf[7, 2] == 0) and np.all(unpack(codes)[7, 32:48] == 0)
+
+
+def test_tensor_scale_is_amax_over_2688(orc):
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal((33, 48)) * 3).astype(F32)
+    amax, st = orc.tensor_scale(x)
+    assert amax == np.max(np.abs(x))
+    assert F32(st) == F32(amax) / F32(6 * 448)
+
+
+# ------------------------------------------------------------------ round trips
+def _representable_tensor(rng, rows, cols, e):
+    """Build x = v(q) * s_b * 2^e with s_t = 2^e exactly: every block holds a
+    +-6 code so its amax is 6 * s_b * s_t, and one block has s_b = 448 so the
+    tensor amax is 2688 * 2^e."""
+    nkb = cols // 16
+    sb = rng.integers(0x08, 0x7F, size=(rows, nkb)).astype(np.uint8)  # normal E4M3
+    sb[0, 0] = 0x7E
+    q = rng.integers(0, 16, size=(rows, cols)).astype(np.uint8)
+    pos = rng.integers(0, 16, size=(rows, nkb))
+    for i in range(rows):
+        for b in range(nkb):
+            q[i, b * 16 + pos[i, b]] = 7 | (8 * rng.integers(0, 2))
+    v = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)[q]
+    s = sb.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    x = v * np.repeat(s, 16, axis=1) * 2.0 ** e
+    return x, q, sb
+
+
+@pytest.mark.parametrize("e", [-20, -3, 0, 5])
+def test_exact_round_trip(orc, e):
+    rng = np.random.default_rng(100 + e)
+    x, q, sb = _representable_tensor(rng, 40, 128, e)
+    x32 = x.astype(F32)
+    assert np.array_equal(x32.astype(np.float64), x)  # representable in binary32
+    codes, sf, st = orc.quantize(x32)
+    assert st == 2.0 ** e
+    np.testing.assert_array_equal(sf, sb)
+    np.testing.assert_array_equal(unpack(codes), q)
+    np.testing.assert_array_equal(orc.dequantize_exact(codes, sf, st), x)
+    # the same tensor in bfloat16 (all values have <= 8 significant bits)
+    bits = bf16_bits(x32)
+    assert np.array_equal(bits_to_f32(bits), x32)
+    codes2, sf2, st2 = orc.quantize(bits)
+    assert st2 == st and np.array_equal(sf2, sf) and np.array_equal(codes2, codes)
+    deq = orc.dequantize(codes, sf, st)
+    np.testing.assert_array_equal(deq, bits)
+
+
+def test_error_bound(orc):
+    """|x - deq(q(x))| <= 1/2 * gap(|q|) * s_b * s_t wherever s_b is a normal
+    E4M3 value and the block did not saturate (gap = 0.5 on [0,2], 1 on
+    [2,4], 2 on [4,6])."""
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(128, 512, generator=g) * torch.exp(torch.randn(128, 1, generator=g))
+    x32 = x.numpy().astype(F32)
+    codes, sf, st = orc.quantize(x32)
+    deq = orc.dequantize_exact(codes, sf, st)
+    q = unpack(codes)
+    mag = np.abs(np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn)
+                 .astype(np.float64)[q])
+    gap = np.where(mag < 2, 0.5, np.where(mag < 4, 1.0, 2.0))
+    # at the top code the step below it is the one that bounds rounding
+    gap = np.where(mag == 6, 2.0, gap)
+    scale = np.repeat(sf.view(ml_dtypes.float8_e4m3fn).astype(np.float64), 16, axis=1) * st
+    normal = np.repeat(sf >= 0x08, 16, axis=1)
+    err = np.abs(x32.astype(np.float64) - deq)
+    bound = 0.5 * gap * scale * (1 + 2.0 ** -20)
+    ok = (err <= bound) | ~normal
+    assert ok.all(), np.argwhere(~ok)[:5]
+    # the recipe keeps the E2M1 argument within 6 * (1 + 2^-4) for normal scales
+    y = np.abs(x32.astype(np.float64)) / scale
+    assert np.max(y[normal]) <= 6 * (1 + 2.0 ** -4)
+
+
+def test_special_cases(orc):
+    z = np.zeros((4, 32), F32)
+    codes, sf, st = orc.quantize(z)
+    assert st == 0 and not sf.any() and not codes.any()
+    x = np.zeros((2, 32), F32)
+    x[0, 0] = -1e-6
+    x[0, 1] = 100.0
+    x[1, 16:32] = -100.0
+    x[0, 2] = -0.0
+    codes, sf, st = orc.quantize(x)
+    q = unpack(codes)
+    assert q[0, 0] == 8  # tiny negative -> -0
+    assert q[0, 1] == 7  # the amax element is +6
+    assert q[0, 2] == 8  # -0 keeps its sign
+    assert np.all(q[1, 16:32] == 15)  # -6
+    assert sf[1, 0] == 0 and np.all(q[1, 0:16] == 0)  # all-zero block
+    with pytest.raises(orc.OracleError):
+        orc.quantize(np.array([[np.nan] + [0] * 15], F32))
+    with pytest.raises(orc.OracleError):
+        orc.quantize(np.array([[np.inf] + [0] * 15], F32))
+    with pytest.raises(orc.OracleError):  # amax too small for the scale domain
+        orc.quantize(np.full((1, 16), 1e-33, F32))
+    with pytest.raises(orc.OracleError):
+        orc.quantize(np.zeros((1, 24), F32))  # cols not a multiple of 16
+
+
+def test_given_tensor_scale_saturates(orc):
+    x = np.linspace(-50, 50, 64, dtype=F32).reshape(2, 32)
+    codes, sf, st = orc.quantize(x, s_t=0.001)
+    assert st == F32(0.001)
+    assert np.all(sf == 0x7E)  # every block needs more than 448
+    q = unpack(codes)
+    assert q[0, 0] == 15 and q[1, 31] == 7
+
+
+def test_dequant_elem_all_codes_and_scales(orc):
+    for s_t in (F32(1.0), F32(0.0123), F32(3.7e-20)):
+        for sb in range(0x7F):
+            for c in range(16):
+                v = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(F32)[c]
+                s = np.array([sb], np.uint8).view(ml_dtypes.float8_e4m3fn).astype(F32)[0]
+                ref = bf16_bits(np.array([F32(v * s) * s_t], F32))[0]
+                assert orc.dequant_elem(c, sb, s_t) == ref
+
+
+def test_size_ratio_matches_pages(orc):
+    facts = json.load(open(GOLD))
+    ratio, tol = facts["kv_compression_ratio"]["value"], facts["kv_compression_ratio"]["tolerance"]
+    rows, cols = 880 * 24, 128  # one latent frame of K
+    bf16_bytes = rows * cols * 2
+    nvfp4_bytes = rows * cols // 2 + rows * cols // facts["block_size"]["value"]
+    assert abs(bf16_bytes / nvfp4_bytes - ratio) < tol
+    # with the 4-byte tensor scale per frame the ratio is unchanged at 2 digits
+    assert abs(bf16_bytes / (nvfp4_bytes + 4) - ratio) < tol
+
+
+# ------------------------------------------------------------------ KV codec
+def test_kv_chunk_is_quantize_of_the_chunk(orc):
+    tpf, heads, hd, nf = 12, 3, 32, 3
+    x = wl.kv_tensor(seed=1, tokens=nf * tpf, heads=heads, head_dim=hd)  # bf16 torch
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    codes, sf, st = orc.kv_quant_chunk(bits.reshape(-1), nf, tpf, heads, hd)
+    c2, s2, st2 = orc.quantize(bits.reshape(nf * tpf * heads, hd))
+    assert np.all(st == st2)
+    np.testing.assert_array_equal(codes.reshape(-1), c2.reshape(-1))
+    np.testing.assert_array_equal(sf.reshape(-1), s2.reshape(-1))
+    # a token stride wider than heads*head_dim reads the same elements
+    stride = heads * hd + 40
+    wide = np.zeros((nf * tpf, stride), np.uint16)
+    wide[:, :heads * hd] = bits.reshape(nf * tpf, heads * hd)
+    wide[:, heads * hd:] = bf16_bits(np.full((1,), 1e4, F32))[0]  # must be ignored
+    c3, s3, st3 = orc.kv_quant_chunk(wide.reshape(-1), nf, tpf, heads, hd, token_stride=stride)
+    assert np.all(st3 == st) and np.array_equal(c3, codes) and np.array_equal(s3, sf)
+
+
+def test_kv_window_is_per_slot_dequant(orc):
+    tpf, heads, hd = 8, 2, 32
+    pool_c, pool_s, pool_t = [], [], []
+    for chunk in range(3):
+        x = wl.kv_tensor(seed=10 + chunk, tokens=2 * tpf, heads=heads, head_dim=hd)
+        bits = x.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+        c, s, t = orc.kv_quant_chunk(bits, 2, tpf, heads, hd)
+        pool_c.append(c); pool_s.append(s); pool_t.append(t)
+    pool_c = np.concatenate(pool_c); pool_s = np.concatenate(pool_s)
+    pool_t = np.concatenate(pool_t)
+    assert pool_t[0] == pool_t[1] and pool_t[2] == pool_t[3]
+    slots = [0, 5, 2, 3]
+    out = orc.kv_dequant_window(pool_c, pool_s, pool_t, slots, tpf, heads, hd)
+    for i, s in enumerate(slots):
+        ref = orc.dequantize(pool_c[s].reshape(tpf * heads, hd // 2),
+                             pool_s[s].reshape(tpf * heads, hd // 16), pool_t[s])
+        np.testing.assert_array_equal(out[i * tpf:(i + 1) * tpf].reshape(tpf * heads, hd), ref)
+    with pytest.raises(orc.OracleError):
+        orc.kv_dequant_window(pool_c, pool_s, pool_t, [6], tpf, heads, hd)
