@@ -1,0 +1,220 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4, the NVFP4 W4A4 path of a causal video DiT on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operations are the inference path the LongLive-2.0 pages describe:
+ *   - NVFP4 tensors: E2M1 4-bit elements, one FP8 (E4M3) scale per block of 16
+ *     elements and one FP32 scale per tensor (neurohive.io LongLive-2.0 article,
+ *     section "Ключевые компоненты LongLive-2.0", NVFP4 paragraph;
+ *     tailorednewshub.com LongLive-2.0 article, section "Entrenamiento NVFP4").
+ *   - W4A4 linear layers: weights and activations both NVFP4, BF16 GEMMs
+ *     replaced by FP4 GEMMs on Blackwell tensor cores (tailorednewshub.com,
+ *     section "Inferencia W4A4 NVFP4").
+ *   - An NVFP4 KV cache quantized in blocks of up to eight latent frames and
+ *     rebuilt to bf16 for windowed attention (hyper.ai LongLive-2.0 summary,
+ *     section "方法" (Method), second paragraph), over a window of 9 local plus
+ *     3 sink frames (171host.com LongLive 2.0 teardown, section 2.2).
+ *
+ * Quantization recipe (the pages name the format only; this library fixes):
+ *   s_t = amax(|x|) / 2688                          (2688 = 6 * 448)
+ *   s_b = E4M3_RNE_sat( amax_block(|x|) / (6 * s_t) )   per 16 elements
+ *   q   = E2M1_RNE_sat( x / (s_b * s_t) )           code 0 when s_b == 0
+ * each step one IEEE binary32 operation rounded to nearest even, in that order.
+ * Dequantization: bf16_RNE( (v(q) * s_b) * s_t ).
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" are CUDA device pointers on the current device;
+ *     "host" pointers are ordinary host memory read before the call returns.
+ *   - The caller owns and allocates every buffer; the library allocates no
+ *     device memory.  It caches per-device kernel attributes only.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument checks happen on the host, before any launch,
+ *     and a rejected call launches nothing.
+ *   - A launch failure returns NVFP4_ERR_CUDA.  Errors found on the device (a
+ *     bounded wait that ran out, a tensor scale outside the recipe's domain) are
+ *     recorded in the workspace status word and returned by
+ *     nvfp4_get_device_status().
+ *   - Inputs must be finite.  The tensor scale must be 0 or lie in
+ *     [2^-108, 2^100] (amax 0 or in about [2^-96.6, 2^111.4]); outside that
+ *     the outputs are unspecified and the status word reads NVFP4_ERR_DOMAIN.
+ *   - The device must be compute capability 10.0 (B200); anything else returns
+ *     NVFP4_ERR_ARCH.  There is no fallback path.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, bad enum */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside what the kernels take */
+  NVFP4_ERR_MISALIGNED = 3,        /* a pointer or stride breaks alignment */
+  NVFP4_ERR_WORKSPACE = 4,         /* workspace missing or too small */
+  NVFP4_ERR_ARCH = 5,              /* current device is not sm_100 */
+  NVFP4_ERR_CUDA = 6,              /* a CUDA runtime call or launch failed */
+  NVFP4_ERR_TIMEOUT = 7,           /* device: a bounded wait ran out */
+  NVFP4_ERR_DOMAIN = 8             /* device: tensor scale outside the domain */
+} nvfp4_status;
+
+/* Element type of a dense input or output tensor. */
+typedef enum { NVFP4_BF16 = 0, NVFP4_FP32 = 1 } nvfp4_dtype;
+
+/* Layout of the E4M3 block scales of an NVFP4 tensor.
+ *   ROWMAJOR: byte [row * (cols/16) + block].
+ *   MMA128x4: the tensor-core layout: 512-byte tiles of 128 rows x 4 blocks,
+ *     tiles ordered row-tile major then block-tile; inside a tile row r, block
+ *     c at (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4.  Rows are padded to a
+ *     multiple of 128 and blocks to a multiple of 4; padding bytes are zero.
+ *     nvfp4_gemm operands must use this layout. */
+typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA128x4 = 1 } nvfp4_sf_layout;
+
+/* An NVFP4 tensor of rows x cols elements (cols a multiple of 16).
+ *   codes: device, [rows][cols/2] bytes; element 2j in the low nibble of
+ *          byte j, element 2j+1 in the high nibble; sign in bit 3 of a nibble.
+ *   sf:    device, nvfp4_sf_bytes(rows, cols, sf_layout) bytes of E4M3 scales.
+ *   s_t:   device, one float (the per-tensor scale).
+ * codes and sf must be 16-byte aligned, s_t 4-byte aligned. */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* sf;
+  float* s_t;
+  int64_t rows;
+  int64_t cols;
+  int32_t sf_layout; /* nvfp4_sf_layout */
+} nvfp4_tensor;
+
+/* The NVFP4 KV cache of one layer: a pool of n_slots frame slots for K and for
+ * V.  One slot holds one latent frame: tokens_per_frame tokens x heads x
+ * head_dim elements, blocks of 16 along head_dim.
+ *   k_codes, v_codes: device, [n_slots][tokens_per_frame*heads*head_dim/2]
+ *   k_sf, v_sf:       device, [n_slots][tokens_per_frame*heads*head_dim/16],
+ *                     row-major ([token][head][head_dim/16]) E4M3 scales
+ *   k_st, v_st:       device, [n_slots] floats: the tensor scale of the chunk
+ *                     that last wrote the slot
+ * Code and scale pools must be 16-byte aligned; head_dim a multiple of 16. */
+typedef struct {
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint8_t* k_sf;
+  uint8_t* v_sf;
+  float* k_st;
+  float* v_st;
+  int32_t n_slots;
+  int32_t tokens_per_frame;
+  int32_t heads;
+  int32_t head_dim;
+} nvfp4_kv_cache;
+
+/* Most frames one kv_quant_chunk call writes (the pages' 8-frame block) and
+ * most slots one kv_dequant_window call reads. */
+#define NVFP4_KV_MAX_CHUNK_FRAMES 8
+#define NVFP4_KV_MAX_WINDOW_SLOTS 256
+
+/* Sizes in bytes of the code and scale buffers of a rows x cols tensor
+ * (0 for invalid arguments). */
+NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
+NVFP4_API size_t nvfp4_sf_bytes(int64_t rows, int64_t cols, int32_t sf_layout);
+
+/* Size of the device workspace the quantizers and the GEMM take: scratch
+ * words for the running amax and CTA counters plus the device status word.
+ * The caller zero-fills it once after allocating it; every call leaves the
+ * scratch words zero again, so it can be reused without clearing.  Calls that
+ * share one workspace must be ordered on the device (one stream, or events):
+ * overlapping calls race on the scratch words. */
+NVFP4_API size_t nvfp4_workspace_bytes(void);
+
+/* Quantize a dense rows x cols tensor to NVFP4 (the recipe above).
+ *   x:      device, bf16 or fp32 (dtype), row stride ld elements (ld >= cols),
+ *           16-byte aligned, ld * element size a multiple of 16 bytes.
+ *   out:    host struct describing device buffers; out->rows/cols must equal
+ *           rows/cols; out->sf_layout picks the scale layout (padding bytes of
+ *           the MMA layout are written as zero).
+ *   s_t_in: NULL to compute s_t from the tensor's amax (two passes over x), or
+ *           a device float holding s_t to use as is (one pass; blocks whose
+ *           amax exceeds 6 * 448 * s_t saturate).
+ *   ws:     device workspace of ws_bytes >= nvfp4_workspace_bytes().
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (cols % 16, more than 2^32 / 8
+ * elements), MISALIGNED, WORKSPACE, ARCH, CUDA; DOMAIN via the status word. */
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                            const nvfp4_tensor* out, const float* s_t_in, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Dequantize an NVFP4 tensor to bf16: out[r * ld + c] = bf16_RNE((v * s_b) * s_t).
+ *   in:  host struct of device buffers, either scale layout.
+ *   out: device bf16, row stride ld >= cols elements, 16-byte aligned,
+ *        ld a multiple of 8.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, ARCH, CUDA. */
+NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64_t ld, void* stream);
+
+/* Block-scaled FP4 x FP4 GEMM, C = A * W^T:
+ *   C[m][n] = (s_tA * s_tW) * sum_k v(qA[m][k]) sA[m][k/16] * v(qW[n][k]) sW[n][k/16]
+ * products and sums on the tensor cores with FP32 accumulation, the scale
+ * product applied once in the epilogue, then rounded to c_dtype.
+ *   A: M x K activations, W: N x K weights (both K-contiguous), both with
+ *      sf_layout == NVFP4_SF_MMA128x4 and the same K.
+ *   Shapes: K a multiple of 64, N a multiple of 256, M >= 1 (any M; tail rows
+ *      are masked).
+ *   C: device, c_dtype (bf16 or fp32), row stride ldc >= N elements, ldc a
+ *      multiple of 8, 16-byte aligned.
+ *   ws: device workspace (status word for the bounded waits).
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, ARCH, CUDA;
+ * TIMEOUT via the status word. */
+NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, int32_t c_dtype,
+                        int64_t ldc, void* ws, size_t ws_bytes, void* stream);
+
+/* Quantize one chunk of n_frames (1..8) new latent frames of K and V into the
+ * cache.  The chunk is one NVFP4 tensor per K and per V: one s_t over the whole
+ * chunk, blocks of 16 along head_dim.  Frame f of the chunk goes to slot
+ * dst_slots[f], whose s_t entry receives the chunk's s_t.
+ *   k, v: device bf16, n_frames * tokens_per_frame tokens, token t at
+ *         k + t * token_stride elements, heads x head_dim contiguous within a
+ *         token (token_stride >= heads * head_dim, a multiple of 8); this reads
+ *         K and V straight out of a fused QKV projection output.
+ *   dst_slots: host, n_frames distinct slot ids in [0, n_slots).
+ *   ws: device workspace.
+ * Errors: INVALID_ARG (slot ids out of range or repeated), UNSUPPORTED_SHAPE,
+ * MISALIGNED, WORKSPACE, ARCH, CUDA; DOMAIN via the status word. */
+NVFP4_API nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const void* k, const void* v,
+                                  int64_t token_stride, const int32_t* dst_slots, int32_t n_frames,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* Rebuild contiguous bf16 K and V for attention from a list of slots, in list
+ * order (for example 3 sink frames followed by the 9 window frames).
+ *   slot_ids: host, n ids in [0, n_slots), 1 <= n <= NVFP4_KV_MAX_WINDOW_SLOTS;
+ *             repeats allowed.
+ *   k_out, v_out: device bf16 [n * tokens_per_frame][heads][head_dim],
+ *                 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, ARCH, CUDA. */
+NVFP4_API nvfp4_status nvfp4_kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slot_ids,
+                                     int32_t n, void* k_out, void* v_out, void* stream);
+
+/* Synchronize `stream`, then read and clear the workspace status word: the
+ * first device-side error recorded since the last call (NVFP4_OK if none). */
+NVFP4_API nvfp4_status nvfp4_get_device_status(void* ws, void* stream);
+
+/* Upper bound, in nanoseconds, on every spin-wait inside the kernels (default
+ * 2 s).  A wait that runs out records NVFP4_ERR_TIMEOUT, drains the kernel's own
+ * copies and tensor-core work in flight, frees its tensor memory and returns.
+ * Applies to launches made after the call (process-wide). */
+NVFP4_API void nvfp4_set_wait_limit_ns(uint64_t ns);
+
+/* Human-readable name of a status code. */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

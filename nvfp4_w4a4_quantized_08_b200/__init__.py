@@ -1,8 +1,12 @@
 """libnvfp4: the NVFP4 W4A4 path of a causal video DiT on B200 (sm_100a).
 
-The compute lives in ``libnvfp4.so`` (hand-written CUDA kernels behind a C ABI
-declared in ``include/nvfp4.h``); the functions here marshal torch tensors'
+The compute lives in ``libnvfp4.so`` (hand-written CUDA kernels behind the C
+ABI declared in ``include/nvfp4.h``); :mod:`.ops` marshals torch tensors'
 device pointers and the current CUDA stream into those calls.  There is no CPU
-fallback: every call raises if the shared library is missing or the device is
-not an sm_100 GPU.
+fallback: every call raises if the shared library is missing, and the library
+refuses any device that is not sm_100.
 """
+from ._native import (BF16, FP32, KV_MAX_CHUNK_FRAMES, KV_MAX_WINDOW_SLOTS, SF_MMA128x4,  # noqa: F401
+                      SF_ROWMAJOR, NVFP4Error)
+from .ops import (KVCache, NVFP4Tensor, codes_bytes, dequantize, device_status, empty,  # noqa: F401
+                  gemm, quantize, set_wait_limit_ns, sf_bytes, workspace)

@@ -1,0 +1,227 @@
+// dequant.cu -- NVFP4 -> bf16 for dense tensors (nvfp4_dequantize) and the
+// KV-cache window rebuild (nvfp4_kv_dequant_window).
+//
+// Every element is bf16_RNE((v(q) * s_b) * s_t): v(q) * s_b is exact in
+// binary32, the product with s_t one rounding, then one bf16 rounding.  A block
+// of 16 elements shares s_b and s_t, so it has only 8 distinct magnitudes: the
+// kernel computes those 8 bf16 values once per block and maps the 16 codes
+// through them with byte permutes, then ORs in each code's sign bit.
+//
+// The window rebuild is the "custom parallel CUDA dequantization kernel" of the
+// hyper.ai LongLive-2.0 summary (section "方法"): it turns the NVFP4 slots of
+// the sink and window frames (171host.com LongLive 2.0 teardown, section 2.2)
+// back into contiguous bf16 K and V for attention.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+constexpr int kDqThreads = 256;
+constexpr int kDqUnroll = 2;
+
+// The 8 bf16 magnitudes of a block, as byte tables for prmt: lo[0..1] hold the
+// low bytes of values 0..7, hi[0..1] the high bytes.
+struct BlockLut {
+  uint32_t lo0, lo1, hi0, hi1;
+};
+
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ BlockLut make_lut(uint32_t sb, float s_t) {
+  const float s = e4m3_to_f32(sb);
+  // (v * s_b) is exact; one rounding for * s_t, one for bf16
+  const float f1 = __fmul_rn(__fmul_rn(0.5f, s), s_t);
+  const float f2 = __fmul_rn(s, s_t);
+  const float f3 = __fmul_rn(__fmul_rn(1.5f, s), s_t);
+  const float f4 = __fmul_rn(__fmul_rn(2.0f, s), s_t);
+  const float f5 = __fmul_rn(__fmul_rn(3.0f, s), s_t);
+  const float f6 = __fmul_rn(__fmul_rn(4.0f, s), s_t);
+  const float f7 = __fmul_rn(__fmul_rn(6.0f, s), s_t);
+  const uint32_t t01 = bf16x2_rn(0.0f, f1), t23 = bf16x2_rn(f2, f3);
+  const uint32_t t45 = bf16x2_rn(f4, f5), t67 = bf16x2_rn(f6, f7);
+  BlockLut l;
+  l.lo0 = prmt(t01, t23, 0x6420);
+  l.hi0 = prmt(t01, t23, 0x7531);
+  l.lo1 = prmt(t45, t67, 0x6420);
+  l.hi1 = prmt(t45, t67, 0x7531);
+  return l;
+}
+
+// 4 codes (nibbles 0..3 of c) -> 4 bf16 in two words.
+__device__ __forceinline__ void lookup4(const BlockLut& l, uint32_t c, uint32_t& o0,
+                                        uint32_t& o1) {
+  const uint32_t sel = c & 0x7777u;
+  const uint32_t lo4 = prmt(l.lo0, l.lo1, sel);
+  const uint32_t hi4 = prmt(l.hi0, l.hi1, sel);
+  o0 = prmt(lo4, hi4, 0x5140) | ((c << 12) & 0x8000u) | ((c << 24) & 0x80000000u);
+  o1 = prmt(lo4, hi4, 0x7362) | ((c << 4) & 0x8000u) | ((c << 16) & 0x80000000u);
+}
+
+// 16 codes (8 bytes) -> 16 bf16 (32 bytes)
+__device__ __forceinline__ void decode_block(const BlockLut& l, uint2 c, uint4& a, uint4& b) {
+  lookup4(l, c.x, a.x, a.y);
+  lookup4(l, c.x >> 16, a.z, a.w);
+  lookup4(l, c.y, b.x, b.y);
+  lookup4(l, c.y >> 16, b.z, b.w);
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t sf_mma_offset_dq(uint32_t row, uint32_t kb, uint32_t ktiles) {
+  return ((row >> 7) * ktiles + (kb >> 2)) * 512u + (row & 31u) * 16u + ((row >> 5) & 3u) * 4u +
+         (kb & 3u);
+}
+
+struct DequantArgs {
+  const uint8_t* codes;
+  const uint8_t* sf;
+  const float* s_t;
+  uint8_t* out;       // bf16
+  int64_t ld;         // elements
+  uint32_t blocks;    // rows * nkb
+  uint32_t nkb;
+  FastDiv nkb_div;
+  uint32_t ktiles;
+};
+
+template <int kSfLayout, bool kContig>
+__global__ void __launch_bounds__(kDqThreads) dequant_kernel(DequantArgs a) {
+  const float s_t = *a.s_t;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < a.blocks;
+       b0 += kDqUnroll * stride) {
+    uint2 c[kDqUnroll];
+    uint32_t sb[kDqUnroll];
+    uint32_t row[kDqUnroll], kb[kDqUnroll];
+#pragma unroll
+    for (int i = 0; i < kDqUnroll; ++i) {
+      const uint32_t b = b0 + i * stride;
+      const bool valid = b < a.blocks;
+      row[i] = fast_div(a.nkb_div, b);
+      kb[i] = b - row[i] * a.nkb;
+      c[i] = valid ? ld_nc_v2(a.codes + 8 * size_t(b)) : make_uint2(0, 0);
+      const uint32_t off = kSfLayout == NVFP4_SF_ROWMAJOR ? b
+                                                         : sf_mma_offset_dq(row[i], kb[i], a.ktiles);
+      sb[i] = valid ? a.sf[off] : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < kDqUnroll; ++i) {
+      const uint32_t b = b0 + i * stride;
+      if (b >= a.blocks) break;
+      const BlockLut l = make_lut(sb[i], s_t);
+      uint4 lo, hi;
+      decode_block(l, c[i], lo, hi);
+      uint8_t* o = kContig ? a.out + 32 * size_t(b)
+                           : a.out + 2 * (int64_t(row[i]) * a.ld + 16 * int64_t(kb[i]));
+      st_v4(o, lo);
+      st_v4(o + 16, hi);
+    }
+  }
+}
+
+struct KvDequantArgs {
+  const uint8_t* codes[2];
+  const uint8_t* sf[2];
+  const float* st[2];
+  uint8_t* out[2];
+  uint32_t blocks;            // n * blocks_per_frame
+  uint32_t blocks_per_frame;
+  FastDiv bpf_div;
+  int32_t slots[NVFP4_KV_MAX_WINDOW_SLOTS];
+};
+
+__global__ void __launch_bounds__(kDqThreads) kv_dequant_kernel(KvDequantArgs a) {
+  const int plane = blockIdx.y;
+  const uint8_t* codes = a.codes[plane];
+  const uint8_t* sfp = a.sf[plane];
+  const float* stp = a.st[plane];
+  uint8_t* out = a.out[plane];
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < a.blocks;
+       b0 += kDqUnroll * stride) {
+    uint2 c[kDqUnroll];
+    uint32_t sb[kDqUnroll];
+    float st[kDqUnroll];
+#pragma unroll
+    for (int i = 0; i < kDqUnroll; ++i) {
+      const uint32_t b = b0 + i * stride;
+      const bool valid = b < a.blocks;
+      const uint32_t j = fast_div(a.bpf_div, valid ? b : 0u);  // position in the slot list
+      const uint32_t bf = b - j * a.blocks_per_frame;
+      const size_t s = size_t(a.slots[j]);
+      const size_t src = s * a.blocks_per_frame + bf;
+      c[i] = valid ? ld_nc_v2(codes + 8 * src) : make_uint2(0, 0);
+      sb[i] = valid ? sfp[src] : 0u;
+      st[i] = valid ? stp[s] : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < kDqUnroll; ++i) {
+      const uint32_t b = b0 + i * stride;
+      if (b >= a.blocks) break;
+      const BlockLut l = make_lut(sb[i], st[i]);
+      uint4 lo, hi;
+      decode_block(l, c[i], lo, hi);
+      st_v4(out + 32 * size_t(b), lo);
+      st_v4(out + 32 * size_t(b) + 16, hi);
+    }
+  }
+}
+
+static int dq_grid(uint32_t blocks, int sm_count) {
+  uint64_t want = (uint64_t(blocks) + kDqThreads * kDqUnroll - 1) / (kDqThreads * kDqUnroll);
+  uint64_t cap = uint64_t(sm_count) * 8;
+  if (want < 1) want = 1;
+  return int(want < cap ? want : cap);
+}
+
+cudaError_t launch_dequantize(const LaunchDequant& d, cudaStream_t st) {
+  DequantArgs a;
+  a.codes = d.codes;
+  a.sf = d.sf;
+  a.s_t = d.s_t;
+  a.out = static_cast<uint8_t*>(d.out);
+  a.ld = d.ld;
+  a.nkb = uint32_t(d.cols / 16);
+  a.blocks = uint32_t(d.rows * a.nkb);
+  a.nkb_div = make_fastdiv(a.nkb);
+  a.ktiles = (a.nkb + 3) / 4;
+  const int grid = dq_grid(a.blocks, d.sm_count);
+  const bool contig = d.ld == d.cols;
+  const bool mma = d.sf_layout == NVFP4_SF_MMA128x4;
+  if (mma) {
+    if (contig) dequant_kernel<NVFP4_SF_MMA128x4, true><<<grid, kDqThreads, 0, st>>>(a);
+    else dequant_kernel<NVFP4_SF_MMA128x4, false><<<grid, kDqThreads, 0, st>>>(a);
+  } else {
+    if (contig) dequant_kernel<NVFP4_SF_ROWMAJOR, true><<<grid, kDqThreads, 0, st>>>(a);
+    else dequant_kernel<NVFP4_SF_ROWMAJOR, false><<<grid, kDqThreads, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_dequant(const LaunchKvDequant& d, cudaStream_t st) {
+  KvDequantArgs a;
+  a.codes[0] = d.k_codes; a.codes[1] = d.v_codes;
+  a.sf[0] = d.k_sf; a.sf[1] = d.v_sf;
+  a.st[0] = d.k_st; a.st[1] = d.v_st;
+  a.out[0] = static_cast<uint8_t*>(d.k_out);
+  a.out[1] = static_cast<uint8_t*>(d.v_out);
+  a.blocks_per_frame = uint32_t(int64_t(d.tpf) * d.heads * d.head_dim / 16);
+  a.bpf_div = make_fastdiv(a.blocks_per_frame);
+  a.blocks = uint32_t(int64_t(d.n) * a.blocks_per_frame);
+  for (int i = 0; i < NVFP4_KV_MAX_WINDOW_SLOTS; ++i) a.slots[i] = i < d.n ? d.slots[i] : 0;
+  const int grid = dq_grid(a.blocks, d.sm_count);
+  kv_dequant_kernel<<<dim3(grid, 2), kDqThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,78 @@
+// kernels.h -- internal launch interface between the C ABI (api.cu) and the
+// kernel files.  Arguments arrive here already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nvfp4.h"
+
+namespace nvfp4 {
+
+struct LaunchQuant {
+  const void* x;
+  int32_t dtype;
+  int64_t rows, cols, ld;
+  uint8_t* codes;
+  uint8_t* sf;
+  int32_t sf_layout;
+  float* s_t_out;
+  const float* s_t_in;
+  void* ws;
+  int sm_count;
+};
+cudaError_t launch_quantize(const LaunchQuant& q, cudaStream_t st);
+
+struct LaunchDequant {
+  const uint8_t* codes;
+  const uint8_t* sf;
+  const float* s_t;
+  int32_t sf_layout;
+  int64_t rows, cols, ld;
+  void* out;
+  int sm_count;
+};
+cudaError_t launch_dequantize(const LaunchDequant& d, cudaStream_t st);
+
+struct LaunchKvQuant {
+  const void* k;
+  const void* v;
+  int64_t token_stride;
+  int32_t n_frames, tpf, heads, head_dim;
+  const int32_t* slots;  // host, n_frames
+  uint8_t *k_codes, *v_codes, *k_sf, *v_sf;
+  float *k_st, *v_st;
+  void* ws;
+  int sm_count;
+};
+cudaError_t launch_kv_quant(const LaunchKvQuant& q, cudaStream_t st);
+
+struct LaunchKvDequant {
+  const uint8_t *k_codes, *v_codes, *k_sf, *v_sf;
+  const float *k_st, *v_st;
+  const int32_t* slots;  // host, n
+  int32_t n, tpf, heads, head_dim;
+  void* k_out;
+  void* v_out;
+  int sm_count;
+};
+cudaError_t launch_kv_dequant(const LaunchKvDequant& d, cudaStream_t st);
+
+struct LaunchGemm {
+  const uint8_t* a_codes;
+  const uint8_t* a_sf;
+  const float* a_st;
+  const uint8_t* w_codes;
+  const uint8_t* w_sf;
+  const float* w_st;
+  int64_t M, N, K;
+  void* c;
+  int32_t c_dtype;
+  int64_t ldc;
+  void* ws;
+  uint64_t wait_limit_ns;
+  int sm_count;
+};
+cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st);
+
+}  // namespace nvfp4

@@ -1,0 +1,106 @@
+"""GPU parity: nvfp4_gemm against the oracle's FP64 reference.
+
+Pass criterion per output element: |y_gpu - y_ref| <= 1e-3 * sum_k |a_k w_k|,
+plus half a bf16 ulp of |y_ref| for bf16 output; y_ref is the binary64 sum of
+the exactly dequantized operands.  The operands themselves are checked
+byte-exact against the oracle's quantization first."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_w4a4_quantized_08_b200 as nv
+from nvfp4_w4a4_quantized_08_b200 import workloads as wl
+
+from _util import assert_gemm_close, assert_quant_equal, bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _operands(orc, a_cpu, w_cpu):
+    qa = nv.quantize(a_cpu.cuda())
+    qw = nv.quantize(w_cpu.cuda())
+    oa = assert_quant_equal(orc, qa, bits(a_cpu), nv.SF_MMA128x4)
+    ow = assert_quant_equal(orc, qw, bits(w_cpu), nv.SF_MMA128x4)
+    return qa, qw, oa, ow
+
+
+def _sample_rows(M, n_random=32, seed=0):
+    rng = np.random.default_rng(seed)
+    tail_start = (M // 128) * 128
+    rows = set(rng.choice(M, size=min(n_random, M), replace=False).tolist())
+    rows.update(range(tail_start, M))  # the whole ragged last tile
+    rows.update([0, M - 1])
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_tiny_gemm_all_elements(orc, out_dtype):
+    """FP4 GEMM M = N = K = 256 on the tiny outlier pair; every element checked."""
+    a, b = wl.tiny_pair()
+    qa, qw, oa, ow = _operands(orc, a, b)
+    y = nv.gemm(qa, qw, out_dtype=out_dtype)
+    y_ref, S = orc.gemm(oa, ow)
+    assert_gemm_close(y.float().cpu().numpy(), y_ref, S, out_dtype == torch.bfloat16)
+    assert nv.device_status() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (100, 256, 128), (128, 512, 192),
+                                   (129, 256, 320), (300, 768, 1024), (77, 256, 4096),
+                                   (513, 1024, 256)])
+def test_small_shapes(orc, M, N, K):
+    g = torch.Generator().manual_seed(M * 31 + N * 7 + K)
+    a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    qa, qw, oa, ow = _operands(orc, a, w)
+    y = nv.gemm(qa, qw, out_dtype=torch.float32)
+    y_ref, S = orc.gemm(oa, ow)
+    assert_gemm_close(y.cpu().numpy(), y_ref, S, False)
+
+
+def test_qkv_projection(orc):
+    """QKV projection: M=2640 (3 frames x 880 tokens), N=9216, K=3072; 32
+    random rows plus the whole 80-row tail tile, all columns."""
+    wk = wl.qkv()
+    qa, qw, oa, ow = _operands(orc, wk.a, wk.w)
+    y = nv.gemm(qa, qw, out_dtype=torch.bfloat16)
+    rows = _sample_rows(wk.a.shape[0])
+    y_ref, S = orc.gemm(oa, ow, rows=rows)
+    assert_gemm_close(y[rows].float().cpu().numpy(), y_ref, S, True)
+
+
+def test_ffn_pair(orc):
+    """FFN up (M=2640, N=14336, K=3072) and down (M=2640, N=3072, K=14336) with the
+    standalone GELU(N(0,1)) down-projection input."""
+    f = wl.ffn()
+    qx, qu, ox, ou = _operands(orc, f.x, f.w_up)
+    y_up = nv.gemm(qx, qu, out_dtype=torch.float32)
+    rows = _sample_rows(f.x.shape[0], n_random=16, seed=1)
+    y_ref, S = orc.gemm(ox, ou, rows=rows)
+    assert_gemm_close(y_up[rows].cpu().numpy(), y_ref, S, False)
+    qh, qd, oh, od = _operands(orc, f.h, f.w_down)
+    y_dn = nv.gemm(qh, qd, out_dtype=torch.bfloat16)
+    rows = _sample_rows(f.h.shape[0], n_random=16, seed=2)
+    y_ref, S = orc.gemm(oh, od, rows=rows)
+    assert_gemm_close(y_dn[rows].float().cpu().numpy(), y_ref, S, True)
+
+
+def test_timeout_path_reports_and_recovers(orc):
+    """A wait limit of 0 ns makes the first wait that is not already satisfied
+    run out: the kernel records NVFP4_ERR_TIMEOUT, drains its copies and MMAs,
+    frees tensor memory and returns; the next call with the normal limit is
+    correct."""
+    g = torch.Generator().manual_seed(8)
+    a = torch.randn(256, 1024, generator=g).to(torch.bfloat16)
+    w = (torch.randn(512, 1024, generator=g) * 0.1).to(torch.bfloat16)
+    qa, qw, oa, ow = _operands(orc, a, w)
+    try:
+        nv.set_wait_limit_ns(0)
+        nv.gemm(qa, qw, out_dtype=torch.float32)
+        st = nv.device_status()
+    finally:
+        nv.set_wait_limit_ns(2_000_000_000)
+    assert st in (0, nv._native.ERR_TIMEOUT)
+    y = nv.gemm(qa, qw, out_dtype=torch.float32)
+    assert nv.device_status() == 0
+    y_ref, S = orc.gemm(oa, ow)
+    assert_gemm_close(y.cpu().numpy(), y_ref, S, False)

@@ -1,0 +1,102 @@
+"""GPU parity: the NVFP4 KV-cache chunk codec (kv_quant_chunk /
+kv_dequant_window) against the CPU oracle, byte for byte."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_w4a4_quantized_08_b200 as nv
+from nvfp4_w4a4_quantized_08_b200 import workloads as wl
+
+from _util import bits, np_u8
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_slots(orc, cache, kv_bits_chunks, tpf, heads, hd):
+    """kv_bits_chunks: list of (slots, k_bits, v_bits, n_frames) written in order."""
+    per = tpf * heads * hd
+    for slots, kb, vb, nf in kv_bits_chunks:
+        for plane, (src, codes_pool, sf_pool, st_pool) in enumerate(
+                [(kb, cache.k_codes, cache.k_sf, cache.k_st),
+                 (vb, cache.v_codes, cache.v_sf, cache.v_st)]):
+            c, s, t = orc.kv_quant_chunk(src, nf, tpf, heads, hd)
+            gc = np_u8(codes_pool)
+            gs = np_u8(sf_pool)
+            gt = st_pool.cpu().numpy()
+            for f, slot in enumerate(slots):
+                np.testing.assert_array_equal(gc[slot], c[f])
+                np.testing.assert_array_equal(gs[slot], s[f])
+                assert np.float32(gt[slot]) == np.float32(t[f])
+    assert per % 16 == 0
+
+
+def test_window_codec_one_layer(orc):
+    """One layer's cache: K, V [10560, 24, 128] (3 sink + 9 window frames of 880
+    tokens), quantized in chunks of 8 and 4 frames, then the 12-slot window
+    (sinks first) rebuilt to bf16."""
+    tpf, heads, hd = wl.TOKENS_PER_FRAME, wl.HEADS, wl.HEAD_DIM
+    k, v = wl.kv_window()
+    cache = nv.KVCache(16, tpf, heads, hd)
+    kg, vg = k.cuda(), v.cuda()
+    # pool slots: frames 0..7 -> slots 4..11, frames 8..11 -> slots 0..3
+    chunks = [(list(range(4, 12)), 0, 8), ([0, 1, 2, 3], 8, 4)]
+    written = []
+    for slots, f0, nf in chunks:
+        t0, t1 = f0 * tpf, (f0 + nf) * tpf
+        cache.quant_chunk(kg[t0:t1], vg[t0:t1], slots)
+        written.append((slots, bits(k[t0:t1]).reshape(-1), bits(v[t0:t1]).reshape(-1), nf))
+    assert nv.device_status() == 0
+    _check_slots(orc, cache, written, tpf, heads, hd)
+    window = [4, 5, 6] + [7, 8, 9, 10, 11, 0, 1, 2, 3]
+    ko, vo = cache.dequant_window(window)
+    pool_c = np_u8(cache.k_codes)
+    pool_s = np_u8(cache.k_sf)
+    pool_t = cache.k_st.cpu().numpy()
+    ref_k = orc.kv_dequant_window(pool_c, pool_s, pool_t, window, tpf, heads, hd)
+    np.testing.assert_array_equal(bits(ko), ref_k)
+    ref_v = orc.kv_dequant_window(np_u8(cache.v_codes), np_u8(cache.v_sf),
+                                  cache.v_st.cpu().numpy(), window, tpf, heads, hd)
+    np.testing.assert_array_equal(bits(vo), ref_v)
+
+
+def test_chunk_from_fused_qkv_output(orc):
+    """K and V read straight out of a [tokens, 3*dim] QKV output (token stride 9216)."""
+    tpf, heads, hd = 880, 24, 128
+    g = torch.Generator().manual_seed(11)
+    qkv = (torch.randn(3 * tpf, 3 * heads * hd, generator=g) * 2).to(torch.bfloat16)
+    cache = nv.KVCache(5, tpf, heads, hd)
+    q = qkv.cuda()
+    d = heads * hd
+    cache.quant_chunk(q[:, d:2 * d], q[:, 2 * d:], [4, 0, 2])
+    kb = bits(qkv[:, d:2 * d].contiguous()).reshape(-1)
+    vb = bits(qkv[:, 2 * d:].contiguous()).reshape(-1)
+    _check_slots(orc, cache, [([4, 0, 2], kb, vb, 3)], tpf, heads, hd)
+
+
+@pytest.mark.parametrize("tpf,heads,hd,nf", [(7, 3, 16, 1), (5, 2, 48, 8), (13, 4, 64, 3),
+                                             (1, 1, 16, 5), (33, 5, 32, 2)])
+def test_small_geometries(orc, tpf, heads, hd, nf):
+    g = torch.Generator().manual_seed(tpf * 100 + hd)
+    k = (torch.randn(nf * tpf, heads, hd, generator=g) * 3).to(torch.bfloat16)
+    v = (torch.randn(nf * tpf, heads, hd, generator=g) * 0.1).to(torch.bfloat16)
+    cache = nv.KVCache(10, tpf, heads, hd)
+    slots = list(range(9, 9 - nf, -1))
+    cache.quant_chunk(k.cuda(), v.cuda(), slots)
+    _check_slots(orc, cache, [(slots, bits(k).reshape(-1), bits(v).reshape(-1), nf)], tpf, heads,
+                 hd)
+    window = [slots[0], slots[-1], slots[0]]  # repeats allowed
+    ko, vo = cache.dequant_window(window)
+    ref = orc.kv_dequant_window(np_u8(cache.k_codes), np_u8(cache.k_sf), cache.k_st.cpu().numpy(),
+                                window, tpf, heads, hd)
+    np.testing.assert_array_equal(bits(ko), ref)
+
+
+def test_bad_slots_rejected_on_host():
+    cache = nv.KVCache(4, 8, 2, 16)
+    k = torch.zeros(16, 2, 16, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(nv.NVFP4Error):
+        cache.quant_chunk(k, k, [0, 4])  # out of range
+    with pytest.raises(nv.NVFP4Error):
+        cache.quant_chunk(k, k, [1, 1])  # repeated
+    with pytest.raises(nv.NVFP4Error):
+        cache.dequant_window([0, -1])
