@@ -1,0 +1,503 @@
+"""Benchmark: one streaming denoise step of a 30-layer 5B-style video DiT on the
+NVFP4 W4A4 path (libnvfp4), on synthetic seeded inputs.
+
+Step (per layer, on a 3-frame chunk of 2640 tokens; dim 3072, 24 heads x 128,
+FFN 14336): quantize the layer input -> QKV GEMM (N=9216) -> kv_quant_chunk of
+the 3 new frames' K and V straight out of the QKV output -> kv_dequant_window
+over 12 cached frames (3 sinks + 9 window) -> quantize the attention-output
+stand-in -> out-proj GEMM -> quantize -> FFN-up GEMM (N=14336) -> requantize
+the intermediate -> FFN-down GEMM; the down output feeds the next layer.
+Attention, norms, residuals and GELU are not part of the NVFP4 path and are not
+run; the attention output is a fixed seeded tensor.  Weights are pre-quantized
+(outside the timed region).  The whole step is captured once as a CUDA graph.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own step (independent chunks, weak
+scaling); ranks only synchronise for the barrier and the max-over-ranks timing.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nvfp4_w4a4_quantized_08_b200 as nv  # noqa: E402
+from nvfp4_w4a4_quantized_08_b200 import workloads as wl  # noqa: E402
+
+M = wl.CHUNK_TOKENS          # 2640
+D = wl.DIM                   # 3072
+F = wl.FFN                   # 14336
+QKV = wl.QKV_N               # 9216
+TPF = wl.TOKENS_PER_FRAME    # 880
+NEW_FRAMES = wl.CHUNK_FRAMES  # 3
+WINDOW = wl.SINK_FRAMES + wl.WINDOW_FRAMES  # 12
+POOL = WINDOW + NEW_FRAMES   # 15 slots per layer
+
+GEMM_SHAPES = {"qkv": (M, QKV, D), "out": (M, D, D), "up": (M, F, D), "down": (M, D, F)}
+GEMM_FLOPS_LAYER = sum(2 * m * n * k for (m, n, k) in GEMM_SHAPES.values())
+Q_BYTES_PER_ELEM = 2 + 0.5625     # bf16 in, 4-bit code + 1/16 E4M3 scale out
+KV_ELEMS_FRAME = TPF * wl.HEADS * wl.HEAD_DIM
+CODEC_BYTES = {
+    "quant_act": 3 * M * D * Q_BYTES_PER_ELEM + 3 * 4,
+    "requant_ffn": M * F * Q_BYTES_PER_ELEM + 4,
+    "kv_quant": 2 * NEW_FRAMES * KV_ELEMS_FRAME * Q_BYTES_PER_ELEM + 2 * 4,
+    "kv_dequant": 2 * WINDOW * KV_ELEMS_FRAME * Q_BYTES_PER_ELEM,
+}
+GEMM_SRC = os.path.join(ROOT, "nvfp4_w4a4_quantized_08_b200", "csrc", "gemm.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "nvfp4_gemm_dit_step_traffic.txt")
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+# ---------------------------------------------------------------- model state
+class Step:
+    """Device state of the denoise step and the per-layer launch sequence."""
+
+    def __init__(self, layers: int, device):
+        self.layers = layers
+        self.dev = device
+        self.w = []       # per layer: (qkv, out, up, down) NVFP4 weights
+        self.cache = []
+        for l in range(layers):
+            ws_bf16 = wl.layer_weights_cuda(l, device=device)
+            self.w.append([nv.quantize(t) for t in ws_bf16])
+            del ws_bf16
+            c = nv.KVCache(POOL, TPF, wl.HEADS, wl.HEAD_DIM, device=device)
+            # prefill the 12 cached frames (sinks + window) with seeded K/V
+            kv = wl.kv_tensor_cuda(seed=l, tokens=WINDOW * TPF, device=device)
+            for f0 in (0, 8):
+                nf = min(8, WINDOW - f0)
+                sl = kv[f0 * TPF:(f0 + nf) * TPF]
+                c.quant_chunk(sl, sl, list(range(f0, f0 + nf)))
+            self.cache.append(c)
+        torch.cuda.synchronize()
+        self.x_in = wl.activations(c=5, i=0).to(device)          # step input
+        self.attn = wl.randn((M, D), 5, 1).to(device)           # attention-output stand-in
+        self.qkv_out = torch.empty(M, QKV, dtype=torch.bfloat16, device=device)
+        self.o_out = torch.empty(M, D, dtype=torch.bfloat16, device=device)
+        self.up_out = torch.empty(M, F, dtype=torch.bfloat16, device=device)
+        self.down_out = [torch.empty(M, D, dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.k_win = torch.empty(WINDOW * TPF, wl.HEADS, wl.HEAD_DIM, dtype=torch.bfloat16,
+                                 device=device)
+        self.v_win = torch.empty_like(self.k_win)
+        self.qa = nv.empty(M, D, device=device)
+        self.qf = nv.empty(M, F, device=device)
+        self.ws = nv.workspace(device)
+        self.new_slots = list(range(WINDOW, POOL))
+        self.window = list(range(wl.SINK_FRAMES)) + \
+            list(range(wl.SINK_FRAMES + NEW_FRAMES, WINDOW)) + self.new_slots
+        assert len(self.window) == WINDOW
+
+    def output(self) -> torch.Tensor:
+        return self.down_out[(self.layers - 1) % 2]
+
+    def run(self, mark=None):
+        """Enqueue one step on the current stream.  `mark(name)` (optional) is
+        called before each launch group and once at the end with None."""
+        mk = mark or (lambda name: None)
+        x = self.x_in
+        for l in range(self.layers):
+            wq, wo, wu, wd = self.w[l]
+            mk("quant_act")
+            nv.quantize(x, out=self.qa, ws=self.ws)
+            mk("gemm_qkv")
+            nv.gemm(self.qa, wq, out=self.qkv_out, ws=self.ws)
+            mk("kv_quant")
+            self.cache[l].quant_chunk(self.qkv_out[:, D:2 * D], self.qkv_out[:, 2 * D:],
+                                      self.new_slots, ws=self.ws)
+            mk("kv_dequant")
+            self.cache[l].dequant_window(self.window, self.k_win, self.v_win)
+            mk("quant_act")
+            nv.quantize(self.attn, out=self.qa, ws=self.ws)
+            mk("gemm_out")
+            nv.gemm(self.qa, wo, out=self.o_out, ws=self.ws)
+            mk("quant_act")
+            nv.quantize(self.o_out, out=self.qa, ws=self.ws)
+            mk("gemm_up")
+            nv.gemm(self.qa, wu, out=self.up_out, ws=self.ws)
+            mk("requant_ffn")
+            nv.quantize(self.up_out, out=self.qf, ws=self.ws)
+            mk("gemm_down")
+            x = self.down_out[l % 2]
+            nv.gemm(self.qf, wd, out=x, ws=self.ws)
+        mk(None)
+
+    # kernels launched per step: quantize = amax + encode (2), gemm 1,
+    # kv_quant = amax + encode (2), kv_dequant 1
+    def launches_per_step(self) -> int:
+        return self.layers * (4 * 2 + 4 * 1 + 2 + 1)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def gemm_traffic_per_launch():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
+    the summary is missing or was taken on a different gemm.cu."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(TRAFFIC_FILE):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("gemm_cu_sha256_16") != src_hash:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch_avg"])
+    except (KeyError, ValueError):
+        return None
+
+
+class CpuSample:
+    """The CPU oracle on a bounded sample of the step: `rows` token rows through
+    one layer's four activation quantizations and four FP64 GEMMs (that layer's
+    weights pre-quantized by the oracle once, not timed), and the K + V codec
+    (quantize + dequantize) of one latent frame."""
+
+    def __init__(self, rows: int = 16, seed_layer: int = 0):
+        import oracle
+        self.oracle = oracle
+        self.cores = oracle.set_threads(0)
+        self.rows = rows
+        if torch.cuda.is_available():
+            wts = [t.cpu() for t in wl.layer_weights_cuda(seed_layer, device="cuda")]
+        else:
+            wts = [wl.weights(n, k, c=5, i=10 + j) for j, (n, k) in
+                   enumerate([(QKV, D), (D, D), (F, D), (D, F)])]
+        self.wq = [oracle.quantize(self.bits(t)) for t in wts]
+        self.x = self.bits(wl.activations(rows=rows, c=5, i=0))
+        self.attn = self.bits(wl.randn((rows, D), 5, 1))
+        self.kv = self.bits(wl.kv_tensor(seed=20, tokens=TPF)).reshape(-1)
+
+    @staticmethod
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    def run(self):
+        """Returns dict(tflops, kv_gbs, cores, sample, seconds)."""
+        o = self.oracle
+
+        def to_bf16_bits(y):
+            return self.bits(torch.from_numpy(np.ascontiguousarray(y, np.float32))
+                             .to(torch.bfloat16))
+
+        t0 = time.perf_counter()
+        o.gemm(o.quantize(self.x), self.wq[0])
+        y, _ = o.gemm(o.quantize(self.attn), self.wq[1])
+        u, _ = o.gemm(o.quantize(to_bf16_bits(y)), self.wq[2])
+        o.gemm(o.quantize(to_bf16_bits(u)), self.wq[3])
+        t_rows = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        ck, sk, tk = o.kv_quant_chunk(self.kv, 1, TPF, wl.HEADS, wl.HEAD_DIM)
+        cv, sv, tv = o.kv_quant_chunk(self.kv, 1, TPF, wl.HEADS, wl.HEAD_DIM)
+        o.kv_dequant_window(ck, sk, tk, [0], TPF, wl.HEADS, wl.HEAD_DIM)
+        o.kv_dequant_window(cv, sv, tv, [0], TPF, wl.HEADS, wl.HEAD_DIM)
+        t_kv = time.perf_counter() - t0
+        flops = self.rows * GEMM_FLOPS_LAYER / M
+        kv_bytes = 2 * 2 * KV_ELEMS_FRAME * Q_BYTES_PER_ELEM
+        desc = (f"CPU oracle, {self.rows} of {M} token rows through one layer (4 activation "
+                f"quantizations + 4 FP64 GEMMs: {flops / 1e9:.2f} GFLOP in {t_rows:.2f} s) and "
+                f"the K+V codec of one 880-token frame ({kv_bytes / 1e6:.1f} MB in {t_kv:.2f} s)")
+        return {"tflops": flops / t_rows / 1e12, "kv_gbs": kv_bytes / t_kv / 1e9,
+                "cores": self.cores, "sample": desc, "seconds": t_rows + t_kv}
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args):
+    rank = env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    res = []
+    sample = CpuSample(rows=args.ref_rows)
+    for i in range(args.warmup + args.steps):
+        r = sample.run()
+        if i >= args.warmup:
+            res.append(r)
+    value = statistics.median(r["tflops"] for r in res)
+    secs = statistics.median(r["seconds"] for r in res)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res[-1]["cores"],
+                         "kind": "oracle", "sample": res[-1]["sample"],
+                         "kv_codec_gbs": statistics.median(r["kv_gbs"] for r in res)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+METRIC = "W4A4 NVFP4 GEMM TFLOP/s & KV quant/dequant GB/s, % of B200 roofline"
+
+
+def config_block(args):
+    return {"workload": f"dit_denoise_step_{args.layers}L_{M}tok", "layers": args.layers,
+            "tokens": M, "dim": D, "ffn": F, "heads": wl.HEADS, "head_dim": wl.HEAD_DIM,
+            "kv_window_frames": WINDOW, "kv_new_frames": NEW_FRAMES,
+            "global_batch": M * max(1, args.gpus), "seq_len": M,
+            "parallelism": f"replica{args.gpus}" if args.gpus > 1 else "single",
+            "l2": "inputs larger than L2 (2.1 GB NVFP4 weights + 1.4 GB KV pools per step)",
+            "stand_ins": "attention output fixed seeded tensor; attention, norm, residual, "
+                         "GELU not run (outside the NVFP4 path)"}
+
+
+def run_ours(args):
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    local = env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    step = Step(args.layers, dev)
+    stream = torch.cuda.Stream(device=dev)
+    # eager warm-up (first calls set kernel attributes), then capture one step
+    with torch.cuda.stream(stream):
+        step.run()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step.run()
+    torch.cuda.synchronize()
+
+    # ---- timed region A: K graph replays, inputs resident in HBM
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    ev0.record(cur)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(cur)
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    flops_step = GEMM_FLOPS_LAYER * args.layers
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+
+    # ---- timed region B: per-kernel CUDA events captured inside a second graph
+    names = []
+    evs = []
+
+    def mark(name):
+        e = torch.cuda.Event(enable_timing=True, external=True)
+        e.record(torch.cuda.current_stream())
+        evs.append(e)
+        names.append(name)
+
+    graph_b = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_b, stream=stream):
+        step.run(mark)
+    torch.cuda.synchronize()
+    per = {}
+    n_prof = max(1, min(args.steps, 5))
+    for _ in range(n_prof):
+        graph_b.replay()
+        torch.cuda.synchronize()
+        for i in range(len(evs) - 1):
+            per.setdefault(names[i], []).append(evs[i].elapsed_time(evs[i + 1]))
+    kernel_ms = {k: sum(v) / n_prof for k, v in per.items()}  # per step
+    gemm_ms = sum(v for k, v in kernel_ms.items() if k.startswith("gemm"))
+    launches = {k: len(v) // n_prof for k, v in per.items()}
+    gemm_launches = sum(v for k, v in launches.items() if k.startswith("gemm"))
+
+    # ---- e2e: host input -> device, step, result -> host
+    h_in = torch.empty(M, D, dtype=torch.bfloat16, pin_memory=True)
+    h_in.copy_(step.x_in.cpu())
+    h_out = torch.empty(M, D, dtype=torch.bfloat16, pin_memory=True)
+    for _ in range(2):
+        step.x_in.copy_(h_in, non_blocking=True)
+        graph.replay()
+        h_out.copy_(step.output(), non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(args.steps):
+        step.x_in.copy_(h_in, non_blocking=True)
+        graph.replay()
+        h_out.copy_(step.output(), non_blocking=True)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = flops_step * world / (ms_e2e / args.steps * 1e-3) / 1e12
+    status = nv.device_status(step.ws)
+
+    peaks, peak_src = measured_peaks()
+    fp4_peak = 4.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    gemm_tflops = flops_step / (gemm_ms * 1e-3) / 1e12
+    codec = {}
+    for k in ("quant_act", "requant_ffn", "kv_quant", "kv_dequant"):
+        b = CODEC_BYTES[k] * args.layers
+        codec[k] = {"ms_per_step": kernel_ms.get(k), "gb_s": b / (kernel_ms[k] * 1e-3) / 1e9,
+                    "frac_hbm": b / (kernel_ms[k] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    kv_bytes = (CODEC_BYTES["kv_quant"] + CODEC_BYTES["kv_dequant"]) * args.layers
+    kv_ms = kernel_ms["kv_quant"] + kernel_ms["kv_dequant"]
+    traffic = gemm_traffic_per_launch()
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            r = CpuSample(rows=args.cpu_rows).run()
+            cpu = {"value": r["tflops"], "unit": "TFLOP/s", "cores": r["cores"],
+                   "kind": "oracle", "sample": r["sample"], "kv_codec_gbs": r["kv_gbs"]}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp4(e2m1)xfp4 -> fp32 acc; codec u8/bf16", "data": "synthetic",
+            "config": config_block(args),
+            "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel",
+                         "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / fp4_peak,
+                         "peak_source": f"{peak_src}: 4 x bf16_tflops_sustained "
+                                        f"({peaks.get('bf16_tflops_sustained')}), nominal "
+                                        "FP4:BF16 dense ratio 4",
+                         "traffic": traffic},
+            "kv_codec": {"gb_s": kv_bytes / (kv_ms * 1e-3) / 1e9,
+                         "frac_hbm": kv_bytes / (kv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "hbm_peak_gbs": peaks["hbm_gbs"]},
+            "codec": codec,
+            "gemm": {"tflops": gemm_tflops, "ms_per_step": gemm_ms,
+                     "launches_per_step": gemm_launches,
+                     "by_shape_ms": {k: v for k, v in kernel_ms.items() if k.startswith("gemm")}},
+            "kernel_ms_per_step": kernel_ms,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * D * 2,
+                    "d2h_bytes_per_step": M * D * 2, "ms_per_step": ms_e2e / args.steps},
+            "gpu_launches": step.launches_per_step() * args.steps,
+            "clocks": clock_info,
+            "device_status": status,
+        }
+        print(json.dumps(line))
+    if dist is not None:
+        del graph, graph_b
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=wl.LAYERS)
+    ap.add_argument("--ref-rows", type=int, default=16, help="rows per reference-arm step")
+    ap.add_argument("--cpu-rows", type=int, default=128, help="rows of the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -11,15 +11,19 @@
 // Structure: one persistent CTA per SM walks 128 x 256 output tiles.
 //   warp 0      TMA producer: 2-D tensor copies of the A and W code tiles
 //               (128-byte K slabs, 128-byte swizzle) and 1-D bulk copies of the
-//               matching 512-byte scale tiles into a 4-stage shared-memory ring.
-//   warp 1      tensor-core issuer: copies each stage's scales into tensor
-//               memory (tcgen05.cp) and issues 4 MMAs of K = 64 per stage; it
-//               also owns the tensor-memory allocation.
+//               matching 512-byte scale tiles into a 3-stage shared-memory ring.
+//   warp 1      tensor-core issuer: per K = 64 step, copies that step's scales
+//               into tensor memory (tcgen05.cp, interleaved with the MMAs) and
+//               issues one MMA; it also owns the tensor-memory allocation.
 //   warps 2..5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
-//               s_tA * s_tW, round to bf16 / fp32, store; masked M tail.
+//               s_tA * s_tW, round to bf16 / fp32, stage in swizzled shared
+//               memory, TMA tensor store (rows past M are clipped by the store).
+// Two accumulators overlap in tensor memory (columns [0,256) and [192,448)):
+// the epilogue reads the 64 shared columns of a tile first and releases them,
+// so the next tile's MMAs run while it drains the other 192 columns.
 // Every spin-wait is bounded (wait_limit_ns).  A wait that runs out records
 // NVFP4_ERR_TIMEOUT, raises a CTA-wide abort flag, and the CTA drains its own
-// copies and MMAs in flight before freeing tensor memory and returning.
+// copies, MMAs and stores in flight before freeing tensor memory and returning.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -34,7 +38,7 @@ namespace gemm {
 constexpr int kBM = 128;          // tile rows (A rows)
 constexpr int kBN = 256;          // tile cols (W rows)
 constexpr int kBKBytes = 128;     // K slab per stage: 128 bytes = 256 FP4 values
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kKSteps = 4;        // MMA K = 64 values = 32 bytes
 constexpr int kABytes = kBM * kBKBytes;      // 16 KB
 constexpr int kBBytes = kBN * kBKBytes;      // 32 KB
@@ -42,19 +46,25 @@ constexpr int kSfaBytes = 4 * 512;           // 4 scale tiles of 128 rows x 4 bl
 constexpr int kSfbBytes = 2 * 4 * 512;       // 2 row tiles of W
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
-constexpr int kAccCols = kBN;                // fp32 accumulator: 128 lanes x 256 cols
-constexpr int kSfColsPerStage = 48;          // SFA 4 x 4 + SFB 4 x 8 columns
+constexpr int kAcc1Col = 192;                // second accumulator; [192,256) shared
+constexpr int kOverlapCols = 256 - kAcc1Col;
+constexpr int kSfCol = 448;                  // per K step j: SFA at +12j, SFB at +12j+4
+constexpr int kStageBufBytes = 32 * 128;     // epilogue staging: 32 rows x 128 bytes
+constexpr int kEpiWarps = 4;
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kABytes;
 constexpr int kOffSfa = kOffB + kStages * kBBytes;
 constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
-constexpr int kOffBar = kOffSfb + kStages * kSfbBytes;
-constexpr int kNumBars = 2 * kStages + 3;    // full[], empty[], acc_full, acc_empty, drain
+constexpr int kOffStage = kOffSfb + kStages * kSfbBytes;            // 1024-aligned
+constexpr int kOffBar = kOffStage + kEpiWarps * 2 * kStageBufBytes;
+constexpr int kNumBars = 2 * kStages + 4;  // full[], empty[], acc_full[2], acc_release, drain
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
 constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
+static_assert(kOffStage % 1024 == 0, "staging buffers need 1024-byte alignment");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // Instruction descriptor, block-scaled kinds: E2M1 A and B (format 1 at bits
 // 7-9 and 10-12), K-major both, N >> 3 at bits 17-22, E4M3 scales (bit 23 = 0),
@@ -77,14 +87,17 @@ __device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
+// Test phase `parity` of `bar`, letting the hardware suspend the thread for up
+// to `hint_ns` while the phase is incomplete (it resumes when the phase completes).
+__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity,
+                                             uint32_t hint_ns = 20000) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -207,13 +220,35 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32
   }
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y,
+                                             uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   map),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most one committed store group still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
 struct Params {
   const uint8_t* a_sf;
   const uint8_t* w_sf;
   const float* a_st;
   const float* w_st;
-  void* c;
-  int64_t ldc;
   uint32_t M, N;
   uint32_t ktiles;   // K / 64
   uint32_t kslabs;   // ceil(K / 256)
@@ -225,16 +260,17 @@ struct Params {
 
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
-                      const __grid_constant__ CUtensorMap map_w, const Params p) {
+                      const __grid_constant__ CUtensorMap map_w,
+                      const __grid_constant__ CUtensorMap map_c, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar_full = sbase + kOffBar;                 // + 8 s
   const uint32_t bar_empty = bar_full + 8 * kStages;         // + 8 s
-  const uint32_t bar_acc_full = bar_empty + 8 * kStages;
-  const uint32_t bar_acc_empty = bar_acc_full + 8;
-  const uint32_t bar_drain = bar_acc_empty + 8;
+  const uint32_t bar_acc_full = bar_empty + 8 * kStages;     // + 8 b
+  const uint32_t bar_acc_release = bar_acc_full + 16;
+  const uint32_t bar_drain = bar_acc_release + 8;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
@@ -247,7 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bar_init(bar_empty + 8 * s, 1);
     }
     bar_init(bar_acc_full, 1);
-    bar_init(bar_acc_empty, 4);
+    bar_init(bar_acc_full + 8, 1);
+    bar_init(bar_acc_release, kEpiWarps);
     bar_init(bar_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -308,31 +345,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, local = 0;
       bool ok = true;
       for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
-        if (!waiter.wait(bar_acc_empty, (local & 1) ^ 1)) break;
+        // the previous tile's epilogue must have read the columns the two
+        // accumulators share (and, before that, all of the tile before it)
+        if (local > 0 && !waiter.wait(bar_acc_release, (local - 1) & 1)) break;
         tc_fence_after();
+        const uint32_t d_tmem = tmem + ((local & 1) ? kAcc1Col : 0);
         for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
           if (!waiter.wait(bar_full + 8 * stage, phase)) { ok = false; break; }
           tc_fence_after();
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
-          const uint32_t sf_col = tmem + kAccCols + kSfColsPerStage * stage;
           const uint32_t sfa_s = sbase + kOffSfa + stage * kSfaBytes;
           const uint32_t sfb_s = sbase + kOffSfb + stage * kSfbBytes;
-          for (uint32_t j = 0; j < nk; ++j) {
-            tc_cp_sf(sf_col + 4 * j, desc_sf(sfa_s + 512 * j));
-            tc_cp_sf(sf_col + 16 + 8 * j, desc_sf(sfb_s + 512 * j));
-            tc_cp_sf(sf_col + 16 + 8 * j + 4, desc_sf(sfb_s + 2048 + 512 * j));
-          }
           const uint32_t a_s = sbase + kOffA + stage * kABytes;
           const uint32_t b_s = sbase + kOffB + stage * kBBytes;
           for (uint32_t j = 0; j < nk; ++j) {
-            tc_mma(tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), kIdesc,
-                   sf_col + 4 * j, sf_col + 16 + 8 * j, (kb | j) != 0);
+            // scales of this K step, then its MMA (tcgen05 ops issue in order)
+            const uint32_t sf_col = tmem + kSfCol + 12 * j;
+            tc_cp_sf(sf_col, desc_sf(sfa_s + 512 * j));
+            tc_cp_sf(sf_col + 4, desc_sf(sfb_s + 512 * j));
+            tc_cp_sf(sf_col + 8, desc_sf(sfb_s + 2048 + 512 * j));
+            tc_mma(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), kIdesc, sf_col,
+                   sf_col + 4, (kb | j) != 0);
           }
           tc_commit(bar_empty + 8 * stage);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(bar_acc_full);
+        tc_commit(bar_acc_full + 8 * (local & 1));
       }
       // drain: every tcgen05 operation this thread issued has completed
       tc_commit(bar_drain);
@@ -340,62 +379,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t quad = uint32_t(warp & 3);
-    const uint32_t row_in_tile = quad * 32 + lane;
+    const uint32_t ew = uint32_t(warp - 2);            // staging buffers of this warp
+    const uint32_t quad = uint32_t(warp & 3);          // tensor-memory lane quadrant
     const float alpha = __fmul_rn(*p.a_st, *p.w_st);
-    uint32_t local = 0;
+    const bool bf16 = p.c_dtype == NVFP4_BF16;
+    const uint32_t chunk_cols = bf16 ? 64 : 32;        // 128-byte rows in staging
+    const uint32_t nchunks = kBN / chunk_cols;
+    const uint32_t overlap_chunks = kOverlapCols / chunk_cols;
+    const uint32_t stage0 = sbase + kOffStage + ew * 2 * kStageBufBytes;
+    uint32_t local = 0, nstore = 0;
     for (uint32_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
       const uint32_t tm = t % p.tiles_m, tn = t / p.tiles_m;
+      const uint32_t buf = local & 1;
       // warp-uniform outcome: tcgen05.ld below is .sync.aligned
-      const bool ok = waiter.wait(bar_acc_full, local & 1);
+      const bool ok = waiter.wait(bar_acc_full + 8 * buf, (local >> 1) & 1);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
-      const uint32_t m = tm * kBM + row_in_tile;
-      const bool row_ok = m < p.M;
-      const uint32_t taddr = tmem + ((quad * 32) << 16);
+      const uint32_t taddr = tmem + ((quad * 32) << 16) + (buf ? kAcc1Col : 0);
+      // the shared columns first: the last 64 of accumulator 0, the first 64 of 1
+      const uint32_t first = buf ? 0 : nchunks - overlap_chunks;
 #pragma unroll 1
-      for (uint32_t cb = 0; cb < kBN / 32; ++cb) {
-        uint32_t r[32];
-        tmem_ld32(taddr + cb * 32, r);
-        if (cb == kBN / 32 - 1) {
+      for (uint32_t i = 0; i < nchunks; ++i) {
+        const uint32_t c = (first + i) % nchunks;
+        uint32_t r[64];
+        tmem_ld32(taddr + c * chunk_cols, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        if (bf16)
+          tmem_ld32(taddr + c * chunk_cols + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        if (i + 1 == overlap_chunks) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) bar_arrive(bar_acc_empty);
+          if (lane == 0) bar_arrive(bar_acc_release);
         }
-        if (row_ok) {
-          const size_t col = size_t(tn) * kBN + cb * 32;
-          if (p.c_dtype == NVFP4_BF16) {
-            uint8_t* dst =
-                static_cast<uint8_t*>(p.c) + (size_t(m) * size_t(p.ldc) + col) * 2;
+        // staging buffer: wait until the store issued two chunks ago has read it
+        const uint32_t sb = stage0 + (nstore & 1) * kStageBufBytes;
+        if (lane == 0) bulk_wait_read_le1();
+        __syncwarp();
+        const uint32_t row = sb + uint32_t(lane) * 128;
+        const uint32_t sw = uint32_t(lane) & 7;  // 128-byte swizzle: 16-byte unit ^ (row % 8)
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 o;
-              uint32_t* ow = &o.x;
+        for (uint32_t u = 0; u < 8; ++u) {
+          uint32_t w0, w1, w2, w3;
+          if (bf16) {
+            float f[8];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float lo = __fmul_rn(__uint_as_float(r[8 * v + 2 * e]), alpha);
-                const float hi = __fmul_rn(__uint_as_float(r[8 * v + 2 * e + 1]), alpha);
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
-                ow[e] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              st_v4(dst + 16 * v, o);
-            }
+            for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(__uint_as_float(r[8 * u + e]), alpha);
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(f[0], f[1]);
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(f[2], f[3]);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(f[4], f[5]);
+            __nv_bfloat162 b3 = __floats2bfloat162_rn(f[6], f[7]);
+            w0 = *reinterpret_cast<uint32_t*>(&b0);
+            w1 = *reinterpret_cast<uint32_t*>(&b1);
+            w2 = *reinterpret_cast<uint32_t*>(&b2);
+            w3 = *reinterpret_cast<uint32_t*>(&b3);
           } else {
-            uint8_t* dst =
-                static_cast<uint8_t*>(p.c) + (size_t(m) * size_t(p.ldc) + col) * 4;
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              uint4 o;
-              o.x = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * v + 0]), alpha));
-              o.y = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * v + 1]), alpha));
-              o.z = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * v + 2]), alpha));
-              o.w = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
-              st_v4(dst + 16 * v, o);
-            }
+            w0 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 0]), alpha));
+            w1 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 1]), alpha));
+            w2 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 2]), alpha));
+            w3 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 3]), alpha));
           }
+          st_shared_v4(row + ((u ^ sw) << 4), w0, w1, w2, w3);
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&map_c, int32_t(tn * kBN + c * chunk_cols), int32_t(tm * kBM + quad * 32),
+                       sb);
+          bulk_commit();
+        }
+        ++nstore;
       }
     }
+    // drain: every store this warp issued has completed
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -425,6 +481,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+// 2-D map over uint8 code rows: box of 128 bytes x box_rows, 128-byte swizzle.
 static bool make_code_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
                           uint32_t box_rows) {
   auto encode = get_encode();
@@ -435,6 +492,25 @@ static bool make_code_map(CUtensorMap* map, const void* base, uint64_t row_bytes
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D map over the output C (rows x cols elements, row stride ldc): box of
+// 128 bytes x 32 rows, 128-byte swizzle (the epilogue's staging layout).
+static bool make_out_map(CUtensorMap* map, void* base, int32_t dtype, uint64_t rows, uint64_t cols,
+                         uint64_t ldc) {
+  auto encode = get_encode();
+  if (!encode) return false;
+  const uint64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ldc * esz};
+  cuuint32_t box[2] = {uint32_t(128 / esz), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, dtype == NVFP4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                      2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -451,17 +527,16 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  CUtensorMap map_a, map_w;
+  CUtensorMap map_a, map_w, map_c;
   if (!make_code_map(&map_a, g.a_codes, uint64_t(g.K / 2), uint64_t(g.M), gemm::kBM) ||
-      !make_code_map(&map_w, g.w_codes, uint64_t(g.K / 2), uint64_t(g.N), gemm::kBN))
+      !make_code_map(&map_w, g.w_codes, uint64_t(g.K / 2), uint64_t(g.N), gemm::kBN) ||
+      !make_out_map(&map_c, g.c, g.c_dtype, uint64_t(g.M), uint64_t(g.N), uint64_t(g.ldc)))
     return cudaErrorInvalidValue;
   gemm::Params p;
   p.a_sf = g.a_sf;
   p.w_sf = g.w_sf;
   p.a_st = g.a_st;
   p.w_st = g.w_st;
-  p.c = g.c;
-  p.ldc = g.ldc;
   p.M = uint32_t(g.M);
   p.N = uint32_t(g.N);
   p.ktiles = uint32_t(g.K / 64);
@@ -473,7 +548,8 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.c_dtype = g.c_dtype;
   const uint32_t tiles = p.tiles_m * p.tiles_n;
   const int grid = int(tiles < uint32_t(g.sm_count) ? tiles : uint32_t(g.sm_count));
-  gemm::nvfp4_gemm_kernel<<<grid, gemm::kThreads, gemm::kSmemBytes, st>>>(map_a, map_w, p);
+  gemm::nvfp4_gemm_kernel<<<grid, gemm::kThreads, gemm::kSmemBytes, st>>>(map_a, map_w, map_c,
+                                                                          p);
   return cudaGetLastError();
 }
 

@@ -125,6 +125,16 @@ def kv_window(c: int = 4):
     return kv_tensor(0, t, c=c), kv_tensor(1, t, c=c)
 
 
+def kv_tensor_cuda(seed: int, tokens: int, heads: int = HEADS, head_dim: int = HEAD_DIM,
+                   device="cuda", c: int = 5) -> torch.Tensor:
+    """kv_tensor's recipe drawn on the GPU (CUDA generator seeded
+    1000 + 100*c + 500 + seed): used to prefill the 30 layers' caches."""
+    g = torch.Generator(device=device).manual_seed(1000 + 100 * c + 500 + seed)
+    sigma = torch.rand(heads, generator=g, device=device) * 3.5 + 0.5
+    x = torch.randn(tokens, heads, head_dim, generator=g, device=device)
+    return (x * sigma[None, :, None]).to(torch.bfloat16)
+
+
 def layer_weights_cuda(layer: int, device="cuda", c: int = 5):
     """The four weight matrices of one DiT layer (QKV, out, up, down) drawn on
     the GPU from a CUDA generator seeded 1000 + 100*c + layer."""
