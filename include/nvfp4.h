@@ -200,6 +200,35 @@ NVFP4_API nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const v
 NVFP4_API nvfp4_status nvfp4_kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slot_ids,
                                      int32_t n, void* k_out, void* v_out, void* stream);
 
+/* Size of the library-owned scratch array behind nvfp4_quantize_noalloc. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+
+/* nvfp4_quantize without a workspace argument, for callers that cannot
+ * allocate device memory when they quantize: code that runs inside a memory
+ * budget whose allocator belongs to someone else (a serving arena, an embedded
+ * runtime), hooks that receive only their input and output buffers, or paths
+ * where a cudaMalloc would synchronize the device at a bad moment.  (The
+ * LongLive-2.0 pages have no counterpart; this is a deployment convenience.)
+ *
+ * Same arguments, recipe and results as nvfp4_quantize, minus ws / ws_bytes.
+ * The scratch words (running amax, CTA counter) live in a fixed array of
+ * NVFP4_NOALLOC_SCRATCH_BYTES bytes of the library's own device memory, which
+ * every GPU that loads the library keeps until the process exits; the call
+ * itself allocates nothing.  The scratch need is constant (20 bytes for any
+ * tensor); a layout that would not fit the array is rejected with
+ * NVFP4_ERR_WORKSPACE, and tensors of 2^32 / 8 or more elements with
+ * NVFP4_ERR_UNSUPPORTED_SHAPE, as in nvfp4_quantize.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Each call first clears the scratch words on `stream`.  All calls on a
+ *     device share the one array, so calls that may overlap on the GPU (other
+ *     streams, other threads) race and must be serialized by the caller.
+ *   - A tensor scale outside the recipe's domain is not reported (there is no
+ *     workspace status word to read); use nvfp4_quantize where that matters. */
+NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void* x, int32_t dtype, int64_t rows,
+                                              int64_t cols, int64_t ld, const nvfp4_tensor* out,
+                                              const float* s_t_in, void* stream);
+
 /* Synchronize `stream`, then read and clear the workspace status word: the
  * first device-side error recorded since the last call (NVFP4_OK if none). */
 NVFP4_API nvfp4_status nvfp4_get_device_status(void* ws, void* stream);

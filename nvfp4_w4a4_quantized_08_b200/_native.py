@@ -34,6 +34,7 @@ EXPORTS = (
     "nvfp4_codes_bytes", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
     "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_quant_chunk", "nvfp4_kv_dequant_window",
     "nvfp4_get_device_status", "nvfp4_set_wait_limit_ns", "nvfp4_status_string",
+    "nvfp4_quantize_noalloc",
 )
 
 
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_workspace_bytes.argtypes = []
         L.nvfp4_quantize.restype = i32
         L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, TP, vp, vp, sz, vp]
+        L.nvfp4_quantize_noalloc.restype = i32
+        L.nvfp4_quantize_noalloc.argtypes = [vp, i32, i64, i64, i64, TP, vp, vp]
         L.nvfp4_dequantize.restype = i32
         L.nvfp4_dequantize.argtypes = [TP, vp, i64, vp]
         L.nvfp4_gemm.restype = i32
