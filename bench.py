@@ -67,6 +67,20 @@ def env_int(name, default):
         return default
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest `value` over all ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own step (weak scaling)."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- model state
 class Step:
     """Device state of the denoise step and the per-layer launch sequence."""
@@ -368,14 +382,10 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     clock_info = clocks.stop()
-    ms_total = ev0.elapsed_time(ev1)
-    if dist is not None:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     ms_step = ms_total / args.steps
     flops_step = GEMM_FLOPS_LAYER * args.layers
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    value = job_throughput(flops_step, world, ms_step)
 
     # ---- timed region B: per-kernel CUDA events captured inside a second graph
     names = []
@@ -422,12 +432,8 @@ def run_ours(args):
         h_out.copy_(step.output(), non_blocking=True)
     e1.record(cur)
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = flops_step * world / (ms_e2e / args.steps * 1e-3) / 1e12
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    e2e_value = job_throughput(flops_step, world, ms_e2e / args.steps)
     status = nv.device_status(step.ws)
 
     peaks, peak_src = measured_peaks()

@@ -90,16 +90,6 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
   return __half2float(__ushort_as_half((unsigned short)(f16x2 & 0xFFFF)));
 }
 
-// Pair product on the packed fp32 pipe: (a0*b0, a1*b1), each rounded to nearest.
-__device__ __forceinline__ void mul2(float a0, float a1, float b0, float b1, float& r0,
-                                     float& r1) {
-  unsigned long long a, b, r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
-}
-
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -110,6 +100,16 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Read-only 16-byte load that may allocate in L1 (for a thread reading a
+// 32-byte block in two halves: the second half then hits L1).
+__device__ __forceinline__ uint4 ld_nc_v4_l1(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;

@@ -61,22 +61,6 @@ __device__ __forceinline__ void lookup4(const BlockLut& l, uint32_t c, uint32_t&
   o1 = prmt(lo4, hi4, 0x7362) | ((c << 4) & 0x8000u) | ((c << 16) & 0x80000000u);
 }
 
-// 16 codes (8 bytes) -> 16 bf16 (32 bytes)
-__device__ __forceinline__ void decode_block(const BlockLut& l, uint2 c, uint4& a, uint4& b) {
-  lookup4(l, c.x, a.x, a.y);
-  lookup4(l, c.x >> 16, a.z, a.w);
-  lookup4(l, c.y, b.x, b.y);
-  lookup4(l, c.y >> 16, b.z, b.w);
-}
-
-__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-               : "=r"(r.x), "=r"(r.y)
-               : "l"(p));
-  return r;
-}
-
 __device__ __forceinline__ uint32_t sf_mma_offset_dq(uint32_t row, uint32_t kb, uint32_t ktiles) {
   return ((row >> 7) * ktiles + (kb >> 2)) * 512u + (row & 31u) * 16u + ((row >> 5) & 3u) * 4u +
          (kb & 3u);
@@ -94,37 +78,41 @@ struct DequantArgs {
   uint32_t ktiles;
 };
 
+// Threads work on half blocks (8 elements: 4 code bytes in, 16 bytes out), so
+// a warp reads 128 contiguous code bytes and writes 512 contiguous bytes; the
+// two threads of a block both build its table.
 template <int kSfLayout, bool kContig>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(DequantArgs a) {
   const float s_t = *a.s_t;
+  const uint32_t halves = 2 * a.blocks;
   const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < a.blocks;
-       b0 += kDqUnroll * stride) {
-    uint2 c[kDqUnroll];
-    uint32_t sb[kDqUnroll];
-    uint32_t row[kDqUnroll], kb[kDqUnroll];
+  for (uint32_t u0 = blockIdx.x * blockDim.x + threadIdx.x; u0 < halves;
+       u0 += kDqUnroll * stride) {
+    uint32_t c[kDqUnroll], sb[kDqUnroll], row[kDqUnroll], kb[kDqUnroll];
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t b = b0 + i * stride;
-      const bool valid = b < a.blocks;
+      const uint32_t u = u0 + i * stride;
+      const bool valid = u < halves;
+      const uint32_t b = u >> 1;
       row[i] = fast_div(a.nkb_div, b);
       kb[i] = b - row[i] * a.nkb;
-      c[i] = valid ? ld_nc_v2(a.codes + 8 * size_t(b)) : make_uint2(0, 0);
+      c[i] = valid ? __ldg(reinterpret_cast<const uint32_t*>(a.codes) + u) : 0u;
       const uint32_t off = kSfLayout == NVFP4_SF_ROWMAJOR ? b
                                                          : sf_mma_offset_dq(row[i], kb[i], a.ktiles);
-      sb[i] = valid ? a.sf[off] : 0u;
+      sb[i] = valid ? __ldg(a.sf + off) : 0u;
     }
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t b = b0 + i * stride;
-      if (b >= a.blocks) break;
+      const uint32_t u = u0 + i * stride;
+      if (u >= halves) break;
       const BlockLut l = make_lut(sb[i], s_t);
-      uint4 lo, hi;
-      decode_block(l, c[i], lo, hi);
-      uint8_t* o = kContig ? a.out + 32 * size_t(b)
-                           : a.out + 2 * (int64_t(row[i]) * a.ld + 16 * int64_t(kb[i]));
-      st_v4(o, lo);
-      st_v4(o + 16, hi);
+      uint4 o;
+      lookup4(l, c[i], o.x, o.y);
+      lookup4(l, c[i] >> 16, o.z, o.w);
+      uint8_t* dst = kContig ? a.out + 16 * size_t(u)
+                             : a.out + 2 * (int64_t(row[i]) * a.ld + 16 * int64_t(kb[i]) +
+                                            8 * int64_t(u & 1));
+      st_v4(dst, o);
     }
   }
 }
@@ -142,43 +130,44 @@ struct KvDequantArgs {
 
 __global__ void __launch_bounds__(kDqThreads) kv_dequant_kernel(KvDequantArgs a) {
   const int plane = blockIdx.y;
-  const uint8_t* codes = a.codes[plane];
-  const uint8_t* sfp = a.sf[plane];
-  const float* stp = a.st[plane];
-  uint8_t* out = a.out[plane];
+  const uint8_t* codes = plane == 0 ? a.codes[0] : a.codes[1];
+  const uint8_t* sfp = plane == 0 ? a.sf[0] : a.sf[1];
+  const float* stp = plane == 0 ? a.st[0] : a.st[1];
+  uint8_t* out = plane == 0 ? a.out[0] : a.out[1];
+  const uint32_t halves = 2 * a.blocks;
   const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < a.blocks;
-       b0 += kDqUnroll * stride) {
-    uint2 c[kDqUnroll];
-    uint32_t sb[kDqUnroll];
+  for (uint32_t u0 = blockIdx.x * blockDim.x + threadIdx.x; u0 < halves;
+       u0 += kDqUnroll * stride) {
+    uint32_t c[kDqUnroll], sb[kDqUnroll];
     float st[kDqUnroll];
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t b = b0 + i * stride;
-      const bool valid = b < a.blocks;
+      const uint32_t u = u0 + i * stride;
+      const bool valid = u < halves;
+      const uint32_t b = u >> 1;
       const uint32_t j = fast_div(a.bpf_div, valid ? b : 0u);  // position in the slot list
       const uint32_t bf = b - j * a.blocks_per_frame;
       const size_t s = size_t(a.slots[j]);
       const size_t src = s * a.blocks_per_frame + bf;
-      c[i] = valid ? ld_nc_v2(codes + 8 * src) : make_uint2(0, 0);
-      sb[i] = valid ? sfp[src] : 0u;
-      st[i] = valid ? stp[s] : 0.0f;
+      c[i] = valid ? __ldg(reinterpret_cast<const uint32_t*>(codes + 8 * src) + (u & 1)) : 0u;
+      sb[i] = valid ? __ldg(sfp + src) : 0u;
+      st[i] = valid ? __ldg(stp + s) : 0.0f;
     }
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t b = b0 + i * stride;
-      if (b >= a.blocks) break;
+      const uint32_t u = u0 + i * stride;
+      if (u >= halves) break;
       const BlockLut l = make_lut(sb[i], st[i]);
-      uint4 lo, hi;
-      decode_block(l, c[i], lo, hi);
-      st_v4(out + 32 * size_t(b), lo);
-      st_v4(out + 32 * size_t(b) + 16, hi);
+      uint4 o;
+      lookup4(l, c[i], o.x, o.y);
+      lookup4(l, c[i] >> 16, o.z, o.w);
+      st_v4(out + 16 * size_t(u), o);
     }
   }
 }
 
 static int dq_grid(uint32_t blocks, int sm_count) {
-  uint64_t want = (uint64_t(blocks) + kDqThreads * kDqUnroll - 1) / (kDqThreads * kDqUnroll);
+  uint64_t want = (2 * uint64_t(blocks) + kDqThreads * kDqUnroll - 1) / (kDqThreads * kDqUnroll);
   uint64_t cap = uint64_t(sm_count) * 8;
   if (want < 1) want = 1;
   return int(want < cap ? want : cap);

@@ -66,13 +66,13 @@ __device__ __forceinline__ void load_unit(const InT* p, bool valid, Raw<InT>& r)
 template <>
 __device__ __forceinline__ void load_unit<__nv_bfloat16>(const __nv_bfloat16* p, bool valid,
                                                          Raw<__nv_bfloat16>& r) {
-  uint4 v = valid ? ld_nc_v4(p) : make_uint4(0, 0, 0, 0);
+  uint4 v = valid ? ld_nc_v4_l1(p) : make_uint4(0, 0, 0, 0);
   r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
 }
 template <>
 __device__ __forceinline__ void load_unit<float>(const float* p, bool valid, Raw<float>& r) {
-  uint4 a = valid ? ld_nc_v4(p) : make_uint4(0, 0, 0, 0);
-  uint4 b = valid ? ld_nc_v4(p + 4) : make_uint4(0, 0, 0, 0);
+  uint4 a = valid ? ld_nc_v4_l1(p) : make_uint4(0, 0, 0, 0);
+  uint4 b = valid ? ld_nc_v4_l1(p + 4) : make_uint4(0, 0, 0, 0);
   r.w[0] = a.x; r.w[1] = a.y; r.w[2] = a.z; r.w[3] = a.w;
   r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
 }
@@ -117,6 +117,25 @@ __device__ __forceinline__ uint32_t unpack_unit<float>(const Raw<float>& r, floa
   return mx;
 }
 
+// ---------------------------------------------------------------- block access
+// A thread handles one 16-element block: two 8-element units.
+template <typename InT, bool kContig>
+__device__ __forceinline__ const InT* block_ptr(const InMap& m, uint32_t b) {
+  if (kContig) return reinterpret_cast<const InT*>(m.x) + 16 * size_t(b);
+  return unit_ptr<InT, kContig>(m, 2 * b);
+}
+
+template <typename InT>
+struct RawBlock {
+  Raw<InT> h[2];
+};
+
+template <typename InT>
+__device__ __forceinline__ void load_block(const InT* p, bool valid, RawBlock<InT>& r) {
+  load_unit<InT>(p, valid, r.h[0]);
+  load_unit<InT>(p + 8, valid, r.h[1]);
+}
+
 // ---------------------------------------------------------------- amax pass
 struct AmaxArgs {
   InMap in[2];
@@ -127,22 +146,24 @@ template <typename InT, bool kContig>
 __global__ void __launch_bounds__(kQuantThreads) amax_kernel(AmaxArgs args) {
   const int plane = blockIdx.y;
   const InMap m = plane == 0 ? args.in[0] : args.in[1];
+  const uint32_t blocks = m.units >> 1;
   uint32_t mx = 0;
   const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t u0 = blockIdx.x * blockDim.x + threadIdx.x; u0 < m.units;
-       u0 += kUnroll * stride) {
-    Raw<InT> raw[kUnroll];
+  for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < blocks;
+       b0 += kUnroll * stride) {
+    RawBlock<InT> raw[kUnroll];
 #pragma unroll
     for (int i = 0; i < kUnroll; ++i) {
-      uint32_t u = u0 + i * stride;
-      bool valid = u < m.units;
-      load_unit<InT>(valid ? unit_ptr<InT, kContig>(m, u) : nullptr, valid, raw[i]);
+      const uint32_t b = b0 + i * stride;
+      const bool valid = b < blocks;
+      load_block<InT>(valid ? block_ptr<InT, kContig>(m, b) : nullptr, valid, raw[i]);
     }
 #pragma unroll
     for (int i = 0; i < kUnroll; ++i) {
       float a[8];
       uint32_t signs;
-      mx = max(mx, unpack_unit<InT>(raw[i], a, signs));
+      mx = max(mx, unpack_unit<InT>(raw[i].h[0], a, signs));
+      mx = max(mx, unpack_unit<InT>(raw[i].h[1], a, signs));
     }
   }
   mx = __reduce_max_sync(0xFFFFFFFFu, mx);
@@ -182,26 +203,34 @@ __device__ __forceinline__ uint32_t block_scale(float amax_b, const ScaleConsts&
   return k.zero ? 0u : sb;
 }
 
-// Magnitude codes of 8 elements (|x| in a) for block scale byte sb.
-__device__ __forceinline__ uint32_t encode_unit(const float a[8], uint32_t sb, float inv_sb,
-                                                const ScaleConsts& k) {
-  float p = __fmul_rn(k.inv_st, inv_sb);
-  float p_lo = __fmul_rn(p, 1.0f - 0x1p-20f);
-  float p_hi = __fmul_rn(p, 1.0f + 0x1p-20f);
-  float l[8], h[8];
+// Magnitude codes of the 16 elements of a block (|x| in a) for block scale
+// byte sb: two 8-code words.
+__device__ __forceinline__ void encode_block(const float a[16], uint32_t sb, float inv_sb,
+                                             const ScaleConsts& k, uint32_t& c0, uint32_t& c1) {
+  const float p = __fmul_rn(k.inv_st, inv_sb);
+  const float p_lo = __fmul_rn(p, 1.0f - 0x1p-20f);
+  const float p_hi = __fmul_rn(p, 1.0f + 0x1p-20f);
+  float l[16], h[16];
 #pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    mul2(a[i], a[i + 1], p_lo, p_lo, l[i], l[i + 1]);
-    mul2(a[i], a[i + 1], p_hi, p_hi, h[i], h[i + 1]);
+  for (int i = 0; i < 16; ++i) {
+    l[i] = __fmul_rn(a[i], p_lo);
+    h[i] = __fmul_rn(a[i], p_hi);
   }
-  uint32_t lo = e2m1x8(l[0], l[1], l[2], l[3], l[4], l[5], l[6], l[7]);
-  uint32_t hi = e2m1x8(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]);
-  if (lo != hi) {
-    float d = __fmul_rn(e4m3_to_f32(sb), k.s_t);
-    lo = e2m1x8(__fdiv_rn(a[0], d), __fdiv_rn(a[1], d), __fdiv_rn(a[2], d), __fdiv_rn(a[3], d),
-                __fdiv_rn(a[4], d), __fdiv_rn(a[5], d), __fdiv_rn(a[6], d), __fdiv_rn(a[7], d));
+  const uint32_t lo0 = e2m1x8(l[0], l[1], l[2], l[3], l[4], l[5], l[6], l[7]);
+  const uint32_t lo1 = e2m1x8(l[8], l[9], l[10], l[11], l[12], l[13], l[14], l[15]);
+  const uint32_t hi0 = e2m1x8(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]);
+  const uint32_t hi1 = e2m1x8(h[8], h[9], h[10], h[11], h[12], h[13], h[14], h[15]);
+  c0 = lo0;
+  c1 = lo1;
+  if ((lo0 != hi0) | (lo1 != hi1)) {
+    // a quotient sits within the bracket of a rounding boundary: take it exactly
+    const float d = __fmul_rn(e4m3_to_f32(sb), k.s_t);
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(a[i], d);
+    c0 = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+    c1 = e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
   }
-  return lo;
 }
 
 __device__ __forceinline__ void fill_inv_table(float* tab) {
@@ -230,15 +259,6 @@ __device__ __forceinline__ void self_clean(uint32_t* ws, int plane) {
   }
 }
 
-// Gather the block-scale bytes of 4 consecutive blocks into lanes 0, 8, 16, 24
-// (lanes 2i and 2i+1 of a warp share block i).
-__device__ __forceinline__ uint32_t gather_sf4(uint32_t sb) {
-  uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
-  uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
-  uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sb, 6);
-  return sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
-}
-
 // ---- dense tensors
 struct QuantArgs {
   InMap in;
@@ -259,6 +279,21 @@ __device__ __forceinline__ uint32_t sf_mma_offset(uint32_t row, uint32_t kb, uin
          (kb & 3u);
 }
 
+// Quantize one block held in `raw`: returns its scale byte and writes its two
+// code words (sign bits included; all +0 when the scale is 0).
+template <typename InT>
+__device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, const float* inv_tab,
+                                                   const ScaleConsts& k, uint2& codes) {
+  float a[16];
+  uint32_t s0, s1;
+  const uint32_t mx = max(unpack_unit<InT>(raw.h[0], a, s0), unpack_unit<InT>(raw.h[1], a + 8, s1));
+  const uint32_t sb = block_scale(__uint_as_float(mx), k);
+  uint32_t c0, c1;
+  encode_block(a, sb, inv_tab[sb & 0x7Fu], k, c0, c1);
+  codes = sb ? make_uint2(c0 | s0, c1 | s1) : make_uint2(0u, 0u);
+  return sb;
+}
+
 template <typename InT, bool kContig, int kSfLayout>
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs args) {
   __shared__ float inv_tab[128];
@@ -272,53 +307,29 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs args) {
   }
   if (in_domain) {
     const ScaleConsts k = make_consts(s_t);
-    const uint32_t lane = threadIdx.x & 31u;
     const uint32_t stride = gridDim.x * blockDim.x;
-    const uint32_t units = args.in.units;
-    for (uint32_t w0 = blockIdx.x * blockDim.x + threadIdx.x - lane; w0 < units;
-         w0 += kUnroll * stride) {
-      Raw<InT> raw[kUnroll];
+    const uint32_t blocks = args.in.units >> 1;
+    for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < blocks;
+         b0 += kUnroll * stride) {
+      RawBlock<InT> raw[kUnroll];
 #pragma unroll
       for (int i = 0; i < kUnroll; ++i) {
-        uint32_t u = w0 + i * stride + lane;
-        bool valid = u < units;
-        load_unit<InT>(valid ? unit_ptr<InT, kContig>(args.in, u) : nullptr, valid, raw[i]);
+        const uint32_t b = b0 + i * stride;
+        const bool valid = b < blocks;
+        load_block<InT>(valid ? block_ptr<InT, kContig>(args.in, b) : nullptr, valid, raw[i]);
       }
 #pragma unroll
       for (int i = 0; i < kUnroll; ++i) {
-        const uint32_t wbase = w0 + i * stride;  // warp-uniform
-        if (wbase >= units) break;
-        const uint32_t u = wbase + lane;
-        const bool valid = u < units;
-        float a[8];
-        uint32_t signs;
-        uint32_t mx = unpack_unit<InT>(raw[i], a, signs);
-        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-        const uint32_t sb = block_scale(__uint_as_float(mx), k);
-        uint32_t code = encode_unit(a, sb, inv_tab[sb & 0x7Fu], k);
-        code = sb ? (code | signs) : 0u;
-        if (valid) reinterpret_cast<uint32_t*>(args.codes)[u] = code;
-        // block scales: block b = u / 2
-        const uint32_t word = gather_sf4(sb);
-        const uint32_t b = u >> 1;
-        const uint32_t bfirst = wbase >> 1;
-        const uint32_t bend = (units + 1) >> 1;
-        const bool whole = bfirst + 16 <= bend;
+        const uint32_t b = b0 + i * stride;
+        if (b >= blocks) break;
+        uint2 codes;
+        const uint32_t sb = quantize_block<InT>(raw[i], inv_tab, k, codes);
+        reinterpret_cast<uint2*>(args.codes)[b] = codes;
         if (kSfLayout == NVFP4_SF_ROWMAJOR) {
-          if (whole) {
-            if ((lane & 7u) == 0) reinterpret_cast<uint32_t*>(args.sf)[b >> 2] = word;
-          } else if (valid && (lane & 1u) == 0) {
-            args.sf[b] = uint8_t(sb);
-          }
+          args.sf[b] = uint8_t(sb);
         } else {
           const uint32_t row = fast_div(args.nkb_div, b);
-          const uint32_t kb = b - row * args.nkb;
-          if (whole && (args.nkb & 3u) == 0) {
-            if ((lane & 7u) == 0)
-              *reinterpret_cast<uint32_t*>(args.sf + sf_mma_offset(row, kb, args.ktiles)) = word;
-          } else if (valid && (lane & 1u) == 0) {
-            args.sf[sf_mma_offset(row, kb, args.ktiles)] = uint8_t(sb);
-          }
+          args.sf[sf_mma_offset(row, b - row * args.nkb, args.ktiles)] = uint8_t(sb);
         }
       }
     }
@@ -354,7 +365,7 @@ struct KvQuantArgs {
   float* st[2];
   uint32_t* ws;
   uint32_t units_per_frame;
-  FastDiv upf_div;
+  FastDiv bpf_div;  // blocks per frame
   int32_t slots[NVFP4_KV_MAX_CHUNK_FRAMES];
   int32_t n_frames;
 };
@@ -373,49 +384,33 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(KvQuantArgs arg
     record_status(args.ws + kWsStatus / 4, NVFP4_ERR_DOMAIN);
   if (in_domain) {
     const InMap m = plane == 0 ? args.in[0] : args.in[1];
+    uint8_t* const codes_pool = plane == 0 ? args.codes[0] : args.codes[1];
+    uint8_t* const sf_pool = plane == 0 ? args.sf[0] : args.sf[1];
     const ScaleConsts k = make_consts(s_t);
-    const uint32_t lane = threadIdx.x & 31u;
     const uint32_t stride = gridDim.x * blockDim.x;
-    const uint32_t units = m.units;
+    const uint32_t blocks = m.units >> 1;
     const uint32_t bpf = args.units_per_frame >> 1;  // blocks per frame
-    for (uint32_t w0 = blockIdx.x * blockDim.x + threadIdx.x - lane; w0 < units;
-         w0 += kUnroll * stride) {
-      Raw<__nv_bfloat16> raw[kUnroll];
+    for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < blocks;
+         b0 += kUnroll * stride) {
+      RawBlock<__nv_bfloat16> raw[kUnroll];
 #pragma unroll
       for (int i = 0; i < kUnroll; ++i) {
-        uint32_t u = w0 + i * stride + lane;
-        bool valid = u < units;
-        load_unit<__nv_bfloat16>(valid ? unit_ptr<__nv_bfloat16, kContig>(m, u) : nullptr, valid,
-                                 raw[i]);
+        const uint32_t b = b0 + i * stride;
+        const bool valid = b < blocks;
+        load_block<__nv_bfloat16>(valid ? block_ptr<__nv_bfloat16, kContig>(m, b) : nullptr,
+                                  valid, raw[i]);
       }
 #pragma unroll
       for (int i = 0; i < kUnroll; ++i) {
-        const uint32_t wbase = w0 + i * stride;
-        if (wbase >= units) break;
-        const uint32_t u = wbase + lane;
-        const bool valid = u < units;
-        float a[8];
-        uint32_t signs;
-        uint32_t mx = unpack_unit<__nv_bfloat16>(raw[i], a, signs);
-        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-        const uint32_t sb = block_scale(__uint_as_float(mx), k);
-        uint32_t code = encode_unit(a, sb, inv_tab[sb & 0x7Fu], k);
-        code = sb ? (code | signs) : 0u;
-        const uint32_t f = fast_div(args.upf_div, valid ? u : 0u);
-        const uint32_t uf = u - f * args.units_per_frame;
+        const uint32_t b = b0 + i * stride;
+        if (b >= blocks) break;
+        uint2 codes;
+        const uint32_t sb = quantize_block<__nv_bfloat16>(raw[i], inv_tab, k, codes);
+        const uint32_t f = fast_div(args.bpf_div, b);
+        const uint32_t bf = b - f * bpf;
         const size_t slot = size_t(args.slots[f]);
-        if (valid)
-          reinterpret_cast<uint32_t*>(args.codes[plane] + slot * args.units_per_frame * 4)[uf] =
-              code;
-        const uint32_t word = gather_sf4(sb);
-        uint8_t* sfp = args.sf[plane] + slot * bpf;
-        const uint32_t bend = (units + 1) >> 1;
-        const bool whole = (wbase >> 1) + 16 <= bend && (bpf & 3u) == 0;
-        if (whole) {
-          if ((lane & 7u) == 0) reinterpret_cast<uint32_t*>(sfp)[(uf >> 1) >> 2] = word;
-        } else if (valid && (lane & 1u) == 0) {
-          sfp[uf >> 1] = uint8_t(sb);
-        }
+        reinterpret_cast<uint2*>(codes_pool + slot * bpf * 8)[bf] = codes;
+        sf_pool[slot * bpf + bf] = uint8_t(sb);
       }
     }
   }
@@ -424,7 +419,8 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(KvQuantArgs arg
 
 // ---------------------------------------------------------------- launchers
 static int grid_for(uint32_t units, int sm_count) {
-  uint64_t want = (uint64_t(units) + kQuantThreads * kUnroll - 1) / (kQuantThreads * kUnroll);
+  const uint64_t blocks = uint64_t(units) / 2;
+  uint64_t want = (blocks + kQuantThreads * kUnroll - 1) / (kQuantThreads * kUnroll);
   uint64_t cap = uint64_t(sm_count) * 8;
   if (want < 1) want = 1;
   return int(want < cap ? want : cap);
@@ -503,7 +499,7 @@ cudaError_t launch_kv_quant(const LaunchKvQuant& q, cudaStream_t st) {
   ka.sf[0] = q.k_sf; ka.sf[1] = q.v_sf;
   ka.st[0] = q.k_st; ka.st[1] = q.v_st;
   ka.units_per_frame = uint32_t(int64_t(q.tpf) * row_elems / 8);
-  ka.upf_div = make_fastdiv(ka.units_per_frame);
+  ka.bpf_div = make_fastdiv(ka.units_per_frame / 2);
   for (int f = 0; f < NVFP4_KV_MAX_CHUNK_FRAMES; ++f) ka.slots[f] = f < q.n_frames ? q.slots[f] : 0;
   ka.n_frames = q.n_frames;
   const int grid = grid_for(aa.in[0].units, q.sm_count);
