@@ -115,6 +115,9 @@ class Step:
         self.qa = nv.empty(M, D, device=device)
         self.qf = nv.empty(M, F, device=device)
         self.ws = nv.workspace(device)
+        # max|C| words handed from a GEMM epilogue to the quantization of its
+        # output: [0] down -> next layer's input, [1] out-proj, [2] FFN up
+        self.amax = torch.zeros(3, dtype=torch.float32, device=device)
         self.new_slots = list(range(WINDOW, POOL))
         self.window = list(range(wl.SINK_FRAMES)) + \
             list(range(wl.SINK_FRAMES + NEW_FRAMES, WINDOW)) + self.new_slots
@@ -128,10 +131,12 @@ class Step:
         called before each launch group and once at the end with None."""
         mk = mark or (lambda name: None)
         x = self.x_in
+        a_x, a_o, a_u = self.amax[0:1], self.amax[1:2], self.amax[2:3]
         for l in range(self.layers):
             wq, wo, wu, wd = self.w[l]
             mk("quant_act")
-            nv.quantize(x, out=self.qa, ws=self.ws)
+            # layer 0's input has no producer in the step: it takes the amax pass
+            nv.quantize(x, out=self.qa, ws=self.ws, amax_in=a_x if l > 0 else None)
             mk("gemm_qkv")
             nv.gemm(self.qa, wq, out=self.qkv_out, ws=self.ws)
             mk("kv_quant")
@@ -142,22 +147,25 @@ class Step:
             mk("quant_act")
             nv.quantize(self.attn, out=self.qa, ws=self.ws)
             mk("gemm_out")
-            nv.gemm(self.qa, wo, out=self.o_out, ws=self.ws)
+            nv.gemm(self.qa, wo, out=self.o_out, ws=self.ws, c_amax=a_o)
             mk("quant_act")
-            nv.quantize(self.o_out, out=self.qa, ws=self.ws)
+            nv.quantize(self.o_out, out=self.qa, ws=self.ws, amax_in=a_o)
             mk("gemm_up")
-            nv.gemm(self.qa, wu, out=self.up_out, ws=self.ws)
+            nv.gemm(self.qa, wu, out=self.up_out, ws=self.ws, c_amax=a_u)
             mk("requant_ffn")
-            nv.quantize(self.up_out, out=self.qf, ws=self.ws)
+            nv.quantize(self.up_out, out=self.qf, ws=self.ws, amax_in=a_u)
             mk("gemm_down")
             x = self.down_out[l % 2]
-            nv.gemm(self.qf, wd, out=x, ws=self.ws)
+            # the last layer's output is not quantized within the step
+            last = l == self.layers - 1
+            nv.gemm(self.qf, wd, out=x, ws=self.ws, c_amax=None if last else a_x)
         mk(None)
 
-    # kernels launched per step: quantize = amax + encode (2), gemm 1,
+    # kernels launched per step: a quantize with its own amax pass 2 (layer 0's
+    # input, the attention output), one fed by a GEMM's c_amax 1, gemm 1,
     # kv_quant = amax + encode (2), kv_dequant 1
     def launches_per_step(self) -> int:
-        return self.layers * (4 * 2 + 4 * 1 + 2 + 1)
+        return self.layers * (2 + 1 + 1 + 1 + 4 * 1 + 2 + 1) + 1
 
 
 # ---------------------------------------------------------------- clocks

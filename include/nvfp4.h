@@ -141,15 +141,20 @@ NVFP4_API size_t nvfp4_workspace_bytes(void);
  *   out:    host struct describing device buffers; out->rows/cols must equal
  *           rows/cols; out->sf_layout picks the scale layout (padding bytes of
  *           the MMA layout are written as zero).
- *   s_t_in: NULL to compute s_t from the tensor's amax (two passes over x), or
- *           a device float holding s_t to use as is (one pass; blocks whose
- *           amax exceeds 6 * 448 * s_t saturate).
+ *   s_t_in: NULL, or a device float holding s_t to use as is (one pass over x;
+ *           blocks whose amax exceeds 6 * 448 * s_t saturate).
+ *   amax_in: NULL, or a device float into which the producer of x has already
+ *           max-accumulated max|x| (nvfp4_gemm's c_amax does this): s_t is
+ *           amax_in / 2688 and the amax pass is skipped.  The call sets
+ *           *amax_in back to 0 when it is done, ready for the next producer.
+ *           With both NULL, s_t comes from an amax pass over x (two passes).
+ *           Passing both is INVALID_ARG.
  *   ws:     device workspace of ws_bytes >= nvfp4_workspace_bytes().
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (cols % 16, more than 2^32 / 8
  * elements), MISALIGNED, WORKSPACE, ARCH, CUDA; DOMAIN via the status word. */
-NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
-                            const nvfp4_tensor* out, const float* s_t_in, void* ws,
-                            size_t ws_bytes, void* stream);
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int32_t dtype, int64_t rows, int64_t cols,
+                                      int64_t ld, const nvfp4_tensor* out, const float* s_t_in,
+                                      float* amax_in, void* ws, size_t ws_bytes, void* stream);
 
 /* Dequantize an NVFP4 tensor to bf16: out[r * ld + c] = bf16_RNE((v * s_b) * s_t).
  *   in:  host struct of device buffers, either scale layout.
@@ -168,11 +173,18 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64
  *      are masked).
  *   C: device, c_dtype (bf16 or fp32), row stride ldc >= N elements, ldc a
  *      multiple of 8, 16-byte aligned.
+ *   c_amax: NULL, or a device float (4-byte aligned) into which the GEMM
+ *      max-accumulates max|C| over the values as stored (after rounding to
+ *      c_dtype), so that nvfp4_quantize(..., amax_in = c_amax, ...) can
+ *      requantize C without an amax pass.  It must hold 0 (or a smaller
+ *      non-negative value) before the call: zero-fill it once; the consuming
+ *      quantize resets it.
  *   ws: device workspace (status word for the bounded waits).
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, ARCH, CUDA;
  * TIMEOUT via the status word. */
-NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, int32_t c_dtype,
-                        int64_t ldc, void* ws, size_t ws_bytes, void* stream);
+NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C,
+                                  int32_t c_dtype, int64_t ldc, float* c_amax, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* Quantize one chunk of n_frames (1..8) new latent frames of K and V into the
  * cache.  The chunk is one NVFP4 tensor per K and per V: one s_t over the whole

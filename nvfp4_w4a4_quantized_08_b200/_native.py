@@ -78,13 +78,13 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_workspace_bytes.restype = sz
         L.nvfp4_workspace_bytes.argtypes = []
         L.nvfp4_quantize.restype = i32
-        L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, TP, vp, vp, sz, vp]
+        L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, TP, vp, vp, vp, sz, vp]
         L.nvfp4_quantize_noalloc.restype = i32
         L.nvfp4_quantize_noalloc.argtypes = [vp, i32, i64, i64, i64, TP, vp, vp]
         L.nvfp4_dequantize.restype = i32
         L.nvfp4_dequantize.argtypes = [TP, vp, i64, vp]
         L.nvfp4_gemm.restype = i32
-        L.nvfp4_gemm.argtypes = [TP, TP, vp, i32, i64, vp, sz, vp]
+        L.nvfp4_gemm.argtypes = [TP, TP, vp, i32, i64, vp, vp, sz, vp]
         L.nvfp4_kv_quant_chunk.restype = i32
         L.nvfp4_kv_quant_chunk.argtypes = [KP, vp, vp, i64, ctypes.POINTER(ctypes.c_int32), i32,
                                            vp, sz, vp]

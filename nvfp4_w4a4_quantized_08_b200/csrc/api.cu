@@ -102,15 +102,17 @@ const char* nvfp4_status_string(nvfp4_status s) {
 }
 
 nvfp4_status nvfp4_quantize(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
-                            const nvfp4_tensor* out, const float* s_t_in, void* ws,
+                            const nvfp4_tensor* out, const float* s_t_in, float* amax_in, void* ws,
                             size_t ws_bytes, void* stream) {
   if (!x || (dtype != NVFP4_BF16 && dtype != NVFP4_FP32)) return NVFP4_ERR_INVALID_ARG;
+  if (s_t_in && amax_in) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_tensor(out);
   if (st != NVFP4_OK) return st;
   if (rows != out->rows || cols != out->cols || ld < cols) return NVFP4_ERR_INVALID_ARG;
   const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
   if (!aligned(x, 16) || (ld * esz) % 16 != 0) return NVFP4_ERR_MISALIGNED;
-  if (s_t_in && !aligned(s_t_in, 4)) return NVFP4_ERR_MISALIGNED;
+  if ((s_t_in && !aligned(s_t_in, 4)) || (amax_in && !aligned(amax_in, 4)))
+    return NVFP4_ERR_MISALIGNED;
   if (!ws || ws_bytes < kWsBytes) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;
   const DeviceInfo dev = current_device();
@@ -126,6 +128,7 @@ nvfp4_status nvfp4_quantize(const void* x, int32_t dtype, int64_t rows, int64_t 
   q.sf_layout = out->sf_layout;
   q.s_t_out = out->s_t;
   q.s_t_in = s_t_in;
+  q.amax_in = amax_in;
   q.ws = ws;
   q.sm_count = dev.sm_count;
   return cuda_status(launch_quantize(q, static_cast<cudaStream_t>(stream)));
@@ -152,7 +155,7 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64_t ld, voi
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, int32_t c_dtype,
-                        int64_t ldc, void* ws, size_t ws_bytes, void* stream) {
+                        int64_t ldc, float* c_amax, void* ws, size_t ws_bytes, void* stream) {
   nvfp4_status st = check_tensor(A);
   if (st != NVFP4_OK) return st;
   st = check_tensor(W);
@@ -166,6 +169,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (ldc < W->rows) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(C, 16) || ldc % 8 != 0) return NVFP4_ERR_MISALIGNED;
+  if (c_amax && !aligned(c_amax, 4)) return NVFP4_ERR_MISALIGNED;
   if (!ws || ws_bytes < kWsBytes) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;
   const DeviceInfo dev = current_device();
@@ -183,6 +187,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
   g.c = C;
   g.c_dtype = c_dtype;
   g.ldc = ldc;
+  g.c_amax = c_amax;
   g.ws = ws;
   g.wait_limit_ns = g_wait_limit_ns.load();
   g.sm_count = dev.sm_count;

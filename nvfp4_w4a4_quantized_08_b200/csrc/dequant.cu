@@ -19,8 +19,8 @@ namespace nvfp4 {
 constexpr int kDqThreads = 256;
 constexpr int kDqUnroll = 2;
 
-// The 8 bf16 magnitudes of a block, as byte tables for prmt: lo[0..1] hold the
-// low bytes of values 0..7, hi[0..1] the high bytes.
+// The 8 bf16 magnitudes of a block, as byte tables for prmt: lo0/lo1 hold the
+// low bytes of values 0..3 / 4..7, hi0/hi1 the high bytes.
 struct BlockLut {
   uint32_t lo0, lo1, hi0, hi1;
 };
@@ -51,14 +51,29 @@ __device__ __forceinline__ BlockLut make_lut(uint32_t sb, float s_t) {
   return l;
 }
 
-// 4 codes (nibbles 0..3 of c) -> 4 bf16 in two words.
-__device__ __forceinline__ void lookup4(const BlockLut& l, uint32_t c, uint32_t& o0,
-                                        uint32_t& o1) {
-  const uint32_t sel = c & 0x7777u;
-  const uint32_t lo4 = prmt(l.lo0, l.lo1, sel);
-  const uint32_t hi4 = prmt(l.hi0, l.hi1, sel);
-  o0 = prmt(lo4, hi4, 0x5140) | ((c << 12) & 0x8000u) | ((c << 24) & 0x80000000u);
-  o1 = prmt(lo4, hi4, 0x7362) | ((c << 4) & 0x8000u) | ((c << 16) & 0x80000000u);
+// 8 codes (nibble i of c = element i) -> 8 bf16 in four words.  Magnitudes
+// come from the block table (byte permutes indexed by the 3 magnitude bits);
+// the sign bits are gathered with one more permute per output word: se holds
+// the signs of the even elements at bit 7 of each byte, so those of the odd
+// elements, and the permute places element 2k's byte at byte 1 and element
+// 2k+1's at byte 3 of word k.
+__device__ __forceinline__ uint4 decode8(const BlockLut& l, uint32_t c) {
+  const uint32_t m = c & 0x77777777u;
+  const uint32_t mh = m >> 16;
+  uint4 o;
+  uint32_t lo4 = prmt(l.lo0, l.lo1, m), hi4 = prmt(l.hi0, l.hi1, m);
+  o.x = prmt(lo4, hi4, 0x5140);
+  o.y = prmt(lo4, hi4, 0x7362);
+  lo4 = prmt(l.lo0, l.lo1, mh);
+  hi4 = prmt(l.hi0, l.hi1, mh);
+  o.z = prmt(lo4, hi4, 0x5140);
+  o.w = prmt(lo4, hi4, 0x7362);
+  const uint32_t se = (c << 4) & 0x80808080u, so = c & 0x80808080u;
+  o.x |= prmt(se, so, 0x4000) & 0x80008000u;
+  o.y |= prmt(se, so, 0x5010) & 0x80008000u;
+  o.z |= prmt(se, so, 0x6020) & 0x80008000u;
+  o.w |= prmt(se, so, 0x7030) & 0x80008000u;
+  return o;
 }
 
 __device__ __forceinline__ uint32_t sf_mma_offset_dq(uint32_t row, uint32_t kb, uint32_t ktiles) {
@@ -78,41 +93,36 @@ struct DequantArgs {
   uint32_t ktiles;
 };
 
-// Threads work on half blocks (8 elements: 4 code bytes in, 16 bytes out), so
-// a warp reads 128 contiguous code bytes and writes 512 contiguous bytes; the
-// two threads of a block both build its table.
+// A thread decodes whole blocks (8 code bytes in, 32 bytes out), kDqUnroll
+// of them per pass with all their loads issued first.  Threads past the end
+// load the last block again and store nothing.
 template <int kSfLayout, bool kContig>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(DequantArgs a) {
   const float s_t = *a.s_t;
-  const uint32_t halves = 2 * a.blocks;
   const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t u0 = blockIdx.x * blockDim.x + threadIdx.x; u0 < halves;
-       u0 += kDqUnroll * stride) {
-    uint32_t c[kDqUnroll], sb[kDqUnroll], row[kDqUnroll], kb[kDqUnroll];
+  for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < a.blocks;
+       b0 += kDqUnroll * stride) {
+    uint2 c[kDqUnroll];
+    uint32_t sb[kDqUnroll], row[kDqUnroll], kb[kDqUnroll];
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t u = u0 + i * stride;
-      const bool valid = u < halves;
-      const uint32_t b = u >> 1;
+      const uint32_t b = min(b0 + i * stride, a.blocks - 1);
       row[i] = fast_div(a.nkb_div, b);
       kb[i] = b - row[i] * a.nkb;
-      c[i] = valid ? __ldg(reinterpret_cast<const uint32_t*>(a.codes) + u) : 0u;
-      const uint32_t off = kSfLayout == NVFP4_SF_ROWMAJOR ? b
-                                                         : sf_mma_offset_dq(row[i], kb[i], a.ktiles);
-      sb[i] = valid ? __ldg(a.sf + off) : 0u;
+      c[i] = __ldg(reinterpret_cast<const uint2*>(a.codes) + b);
+      const uint32_t off =
+          kSfLayout == NVFP4_SF_ROWMAJOR ? b : sf_mma_offset_dq(row[i], kb[i], a.ktiles);
+      sb[i] = __ldg(a.sf + off);
     }
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t u = u0 + i * stride;
-      if (u >= halves) break;
+      const uint32_t b = b0 + i * stride;
+      if (b >= a.blocks) break;
       const BlockLut l = make_lut(sb[i], s_t);
-      uint4 o;
-      lookup4(l, c[i], o.x, o.y);
-      lookup4(l, c[i] >> 16, o.z, o.w);
-      uint8_t* dst = kContig ? a.out + 16 * size_t(u)
-                             : a.out + 2 * (int64_t(row[i]) * a.ld + 16 * int64_t(kb[i]) +
-                                            8 * int64_t(u & 1));
-      st_v4(dst, o);
+      uint8_t* dst = kContig ? a.out + 32 * size_t(b)
+                             : a.out + 2 * (int64_t(row[i]) * a.ld + 16 * int64_t(kb[i]));
+      st_v4(dst, decode8(l, c[i].x));
+      st_v4(dst + 16, decode8(l, c[i].y));
     }
   }
 }
@@ -134,41 +144,45 @@ __global__ void __launch_bounds__(kDqThreads) kv_dequant_kernel(KvDequantArgs a)
   const uint8_t* sfp = plane == 0 ? a.sf[0] : a.sf[1];
   const float* stp = plane == 0 ? a.st[0] : a.st[1];
   uint8_t* out = plane == 0 ? a.out[0] : a.out[1];
-  const uint32_t halves = 2 * a.blocks;
   const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t u0 = blockIdx.x * blockDim.x + threadIdx.x; u0 < halves;
-       u0 += kDqUnroll * stride) {
-    uint32_t c[kDqUnroll], sb[kDqUnroll];
+  for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < a.blocks;
+       b0 += kDqUnroll * stride) {
+    uint2 c[kDqUnroll];
+    uint32_t sb[kDqUnroll];
     float st[kDqUnroll];
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t u = u0 + i * stride;
-      const bool valid = u < halves;
-      const uint32_t b = u >> 1;
-      const uint32_t j = fast_div(a.bpf_div, valid ? b : 0u);  // position in the slot list
+      const uint32_t b = min(b0 + i * stride, a.blocks - 1);
+      const uint32_t j = fast_div(a.bpf_div, b);  // position in the slot list
       const uint32_t bf = b - j * a.blocks_per_frame;
       const size_t s = size_t(a.slots[j]);
       const size_t src = s * a.blocks_per_frame + bf;
-      c[i] = valid ? __ldg(reinterpret_cast<const uint32_t*>(codes + 8 * src) + (u & 1)) : 0u;
-      sb[i] = valid ? __ldg(sfp + src) : 0u;
-      st[i] = valid ? __ldg(stp + s) : 0.0f;
+      c[i] = __ldg(reinterpret_cast<const uint2*>(codes) + src);
+      sb[i] = __ldg(sfp + src);
+      st[i] = __ldg(stp + s);
     }
 #pragma unroll
     for (int i = 0; i < kDqUnroll; ++i) {
-      const uint32_t u = u0 + i * stride;
-      if (u >= halves) break;
+      const uint32_t b = b0 + i * stride;
+      if (b >= a.blocks) break;
       const BlockLut l = make_lut(sb[i], st[i]);
-      uint4 o;
-      lookup4(l, c[i], o.x, o.y);
-      lookup4(l, c[i] >> 16, o.z, o.w);
-      st_v4(out + 16 * size_t(u), o);
+      st_v4(out + 32 * size_t(b), decode8(l, c[i].x));
+      st_v4(out + 32 * size_t(b) + 16, decode8(l, c[i].y));
     }
   }
 }
 
-static int dq_grid(uint32_t blocks, int sm_count) {
-  uint64_t want = (2 * uint64_t(blocks) + kDqThreads * kDqUnroll - 1) / (kDqThreads * kDqUnroll);
-  uint64_t cap = uint64_t(sm_count) * 8;
+// CTAs per plane: kDqUnroll blocks per thread, at most one resident wave.
+template <typename Kernel>
+static int dq_grid(Kernel kernel, uint32_t blocks, int sm_count, int planes) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kDqThreads, 0) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  uint64_t want = (uint64_t(blocks) + kDqThreads * kDqUnroll - 1) / (kDqThreads * kDqUnroll);
+  uint64_t cap = uint64_t(per_sm) * uint64_t(sm_count) / uint64_t(planes);
+  if (cap < 1) cap = 1;
   if (want < 1) want = 1;
   return int(want < cap ? want : cap);
 }
@@ -184,15 +198,17 @@ cudaError_t launch_dequantize(const LaunchDequant& d, cudaStream_t st) {
   a.blocks = uint32_t(d.rows * a.nkb);
   a.nkb_div = make_fastdiv(a.nkb);
   a.ktiles = (a.nkb + 3) / 4;
-  const int grid = dq_grid(a.blocks, d.sm_count);
   const bool contig = d.ld == d.cols;
   const bool mma = d.sf_layout == NVFP4_SF_MMA128x4;
+  auto launch = [&](auto kernel) {
+    kernel<<<dq_grid(kernel, a.blocks, d.sm_count, 1), kDqThreads, 0, st>>>(a);
+  };
   if (mma) {
-    if (contig) dequant_kernel<NVFP4_SF_MMA128x4, true><<<grid, kDqThreads, 0, st>>>(a);
-    else dequant_kernel<NVFP4_SF_MMA128x4, false><<<grid, kDqThreads, 0, st>>>(a);
+    if (contig) launch(dequant_kernel<NVFP4_SF_MMA128x4, true>);
+    else launch(dequant_kernel<NVFP4_SF_MMA128x4, false>);
   } else {
-    if (contig) dequant_kernel<NVFP4_SF_ROWMAJOR, true><<<grid, kDqThreads, 0, st>>>(a);
-    else dequant_kernel<NVFP4_SF_ROWMAJOR, false><<<grid, kDqThreads, 0, st>>>(a);
+    if (contig) launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true>);
+    else launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false>);
   }
   return cudaGetLastError();
 }
@@ -208,7 +224,7 @@ cudaError_t launch_kv_dequant(const LaunchKvDequant& d, cudaStream_t st) {
   a.bpf_div = make_fastdiv(a.blocks_per_frame);
   a.blocks = uint32_t(int64_t(d.n) * a.blocks_per_frame);
   for (int i = 0; i < NVFP4_KV_MAX_WINDOW_SLOTS; ++i) a.slots[i] = i < d.n ? d.slots[i] : 0;
-  const int grid = dq_grid(a.blocks, d.sm_count);
+  const int grid = dq_grid(kv_dequant_kernel, a.blocks, d.sm_count, 2);
   kv_dequant_kernel<<<dim3(grid, 2), kDqThreads, 0, st>>>(a);
   return cudaGetLastError();
 }

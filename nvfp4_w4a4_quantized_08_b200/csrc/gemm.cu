@@ -254,6 +254,7 @@ struct Params {
   uint32_t kslabs;   // ceil(K / 256)
   uint32_t tiles_m, tiles_n;
   uint32_t* status;
+  uint32_t* c_amax;  // float bits of max|C| (atomicMax), or null
   uint64_t wait_limit_ns;
   int32_t c_dtype;
 };
@@ -388,8 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t overlap_chunks = kOverlapCols / chunk_cols;
     const uint32_t stage0 = sbase + kOffStage + ew * 2 * kStageBufBytes;
     uint32_t local = 0, nstore = 0;
+    // running max of |stored value| as magnitude bits: two bf16 halves, or fp32
+    uint32_t vmax = 0;
+    const bool want_max = p.c_amax != nullptr;
     for (uint32_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
       const uint32_t tm = t % p.tiles_m, tn = t / p.tiles_m;
+      // accumulator lanes past the last row of C hold zeros; leave them out anyway
+      const bool row_live = want_max && tm * kBM + quad * 32 + uint32_t(lane) < p.M;
       const uint32_t buf = local & 1;
       // warp-uniform outcome: tcgen05.ld below is .sync.aligned
       const bool ok = waiter.wait(bar_acc_full + 8 * buf, (local >> 1) & 1);
@@ -431,11 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             w1 = *reinterpret_cast<uint32_t*>(&b1);
             w2 = *reinterpret_cast<uint32_t*>(&b2);
             w3 = *reinterpret_cast<uint32_t*>(&b3);
+            if (row_live)
+              vmax = __vmaxu2(__vmaxu2(vmax, __vmaxu2(w0 & 0x7FFF7FFFu, w1 & 0x7FFF7FFFu)),
+                              __vmaxu2(w2 & 0x7FFF7FFFu, w3 & 0x7FFF7FFFu));
           } else {
             w0 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 0]), alpha));
             w1 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 1]), alpha));
             w2 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 2]), alpha));
             w3 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 3]), alpha));
+            if (row_live)
+              vmax = max(max(vmax, max(w0 & 0x7FFFFFFFu, w1 & 0x7FFFFFFFu)),
+                         max(w2 & 0x7FFFFFFFu, w3 & 0x7FFFFFFFu));
           }
           st_shared_v4(row + ((u ^ sw) << 4), w0, w1, w2, w3);
         }
@@ -448,6 +460,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++nstore;
       }
+    }
+    if (want_max) {
+      // fold the bf16 halves into fp32 bits (bf16 bits << 16 is the same value)
+      const uint32_t bits = bf16 ? (max(vmax & 0xFFFFu, vmax >> 16) << 16) : vmax;
+      const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, bits);
+      if (lane == 0 && wmax != 0) atomicMax(p.c_amax, wmax);
     }
     // drain: every store this warp issued has completed
     if (lane == 0) bulk_wait_all();
@@ -544,6 +562,7 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.tiles_m = uint32_t((g.M + gemm::kBM - 1) / gemm::kBM);
   p.tiles_n = uint32_t(g.N / gemm::kBN);
   p.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(g.ws) + kWsStatus);
+  p.c_amax = reinterpret_cast<uint32_t*>(g.c_amax);
   p.wait_limit_ns = g.wait_limit_ns;
   p.c_dtype = g.c_dtype;
   const uint32_t tiles = p.tiles_m * p.tiles_n;

@@ -18,6 +18,7 @@ struct LaunchQuant {
   int32_t sf_layout;
   float* s_t_out;
   const float* s_t_in;
+  float* amax_in;  // producer-accumulated amax (consumed and reset), or NULL
   void* ws;
   int sm_count;
 };
@@ -69,6 +70,7 @@ struct LaunchGemm {
   void* c;
   int32_t c_dtype;
   int64_t ldc;
+  float* c_amax;  // max|C| accumulator, or NULL
   void* ws;
   uint64_t wait_limit_ns;
   int sm_count;

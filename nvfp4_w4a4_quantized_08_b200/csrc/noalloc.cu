@@ -85,6 +85,7 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int32_t dtype, int
   q.sf_layout = out->sf_layout;
   q.s_t_out = out->s_t;
   q.s_t_in = s_t_in;
+  q.amax_in = nullptr;
   q.ws = scratch;
   q.sm_count = sms;
   return launch_quantize(q, st) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

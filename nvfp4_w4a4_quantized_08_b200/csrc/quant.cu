@@ -26,7 +26,7 @@
 namespace nvfp4 {
 
 constexpr int kQuantThreads = 256;
-constexpr int kUnroll = 2;
+constexpr int kAmaxUnroll = 4;  // blocks a thread of the amax pass loads at once
 
 // Where the 8-element units of an input plane live.
 struct InMap {
@@ -61,18 +61,21 @@ struct Raw<float> {
   uint32_t w[8];
 };
 
+// Loads are unconditional: a thread past the end loads the last block again
+// (always a valid address) and discards it, which costs less than a branch
+// around each load.
 template <typename InT>
-__device__ __forceinline__ void load_unit(const InT* p, bool valid, Raw<InT>& r);
+__device__ __forceinline__ void load_unit(const InT* p, Raw<InT>& r);
 template <>
-__device__ __forceinline__ void load_unit<__nv_bfloat16>(const __nv_bfloat16* p, bool valid,
+__device__ __forceinline__ void load_unit<__nv_bfloat16>(const __nv_bfloat16* p,
                                                          Raw<__nv_bfloat16>& r) {
-  uint4 v = valid ? ld_nc_v4_l1(p) : make_uint4(0, 0, 0, 0);
+  uint4 v = ld_nc_v4_l1(p);
   r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
 }
 template <>
-__device__ __forceinline__ void load_unit<float>(const float* p, bool valid, Raw<float>& r) {
-  uint4 a = valid ? ld_nc_v4_l1(p) : make_uint4(0, 0, 0, 0);
-  uint4 b = valid ? ld_nc_v4_l1(p + 4) : make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ void load_unit<float>(const float* p, Raw<float>& r) {
+  uint4 a = ld_nc_v4_l1(p);
+  uint4 b = ld_nc_v4_l1(p + 4);
   r.w[0] = a.x; r.w[1] = a.y; r.w[2] = a.z; r.w[3] = a.w;
   r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
 }
@@ -131,9 +134,9 @@ struct RawBlock {
 };
 
 template <typename InT>
-__device__ __forceinline__ void load_block(const InT* p, bool valid, RawBlock<InT>& r) {
-  load_unit<InT>(p, valid, r.h[0]);
-  load_unit<InT>(p + 8, valid, r.h[1]);
+__device__ __forceinline__ void load_block(const InT* p, RawBlock<InT>& r) {
+  load_unit<InT>(p, r.h[0]);
+  load_unit<InT>(p + 8, r.h[1]);
 }
 
 // ---------------------------------------------------------------- amax pass
@@ -150,16 +153,15 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(AmaxArgs args) {
   uint32_t mx = 0;
   const uint32_t stride = gridDim.x * blockDim.x;
   for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < blocks;
-       b0 += kUnroll * stride) {
-    RawBlock<InT> raw[kUnroll];
+       b0 += kAmaxUnroll * stride) {
+    RawBlock<InT> raw[kAmaxUnroll];
 #pragma unroll
-    for (int i = 0; i < kUnroll; ++i) {
+    for (int i = 0; i < kAmaxUnroll; ++i) {
       const uint32_t b = b0 + i * stride;
-      const bool valid = b < blocks;
-      load_block<InT>(valid ? block_ptr<InT, kContig>(m, b) : nullptr, valid, raw[i]);
+      load_block<InT>(block_ptr<InT, kContig>(m, min(b, blocks - 1)), raw[i]);
     }
 #pragma unroll
-    for (int i = 0; i < kUnroll; ++i) {
+    for (int i = 0; i < kAmaxUnroll; ++i) {
       float a[8];
       uint32_t signs;
       mx = max(mx, unpack_unit<InT>(raw[i].h[0], a, signs));
@@ -195,42 +197,87 @@ __device__ __forceinline__ ScaleConsts make_consts(float s_t) {
   return k;
 }
 
+// The exact fallbacks below are out of line on purpose: inlined, the compiler
+// predicates them into the common path, which then issues their divisions for
+// every block.  A call is always a real branch.  They are not rare enough to
+// ignore: bf16 inputs and a tensor scale derived from a bf16 amax put 0.1 to
+// 1 percent of quotients exactly on (or within 2^-20 of) a rounding boundary,
+// so a few percent of blocks, and most warps, meet one.
+__device__ __noinline__ uint32_t e4m3_of_quotient(float a, float c) {
+  return e4m3x2(0.0f, __fdiv_rn(a, c)) & 0xFFu;
+}
+
+__device__ __noinline__ uint32_t e2m1_of_quotient(float a, float d) {
+  const float y = __fdiv_rn(a, d);
+  return e2m1x8(y, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f) & 0xFu;
+}
+
 // E4M3 block scale of a block with amax amax_b: E4M3_RNE_sat(amax_b / c).
 __device__ __forceinline__ uint32_t block_scale(float amax_b, const ScaleConsts& k) {
   uint32_t two = e4m3x2(__fmul_rn(amax_b, k.rc_hi), __fmul_rn(amax_b, k.rc_lo));
   uint32_t sb = two & 0xFFu;
-  if (sb != (two >> 8)) sb = e4m3x2(0.0f, __fdiv_rn(amax_b, k.c)) & 0xFFu;
+  if (sb != (two >> 8)) sb = e4m3_of_quotient(amax_b, k.c);
   return k.zero ? 0u : sb;
 }
 
 // Magnitude codes of the 16 elements of a block (|x| in a) for block scale
-// byte sb: two 8-code words.
-__device__ __forceinline__ void encode_block(const float a[16], uint32_t sb, float inv_sb,
-                                             const ScaleConsts& k, uint32_t& c0, uint32_t& c1) {
+// byte sb from the two bracketing products: lo/hi code words of each half.
+// Nibbles where lo and hi differ need the exact quotient.
+__device__ __forceinline__ void bracket_codes(const float a[16], float inv_sb,
+                                              const ScaleConsts& k, uint32_t lo[2],
+                                              uint32_t hi[2]) {
   const float p = __fmul_rn(k.inv_st, inv_sb);
   const float p_lo = __fmul_rn(p, 1.0f - 0x1p-20f);
   const float p_hi = __fmul_rn(p, 1.0f + 0x1p-20f);
+  // products on the packed fp32 pipe, two elements per instruction
   float l[16], h[16];
+  const float2 plo2 = make_float2(p_lo, p_lo), phi2 = make_float2(p_hi, p_hi);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    l[i] = __fmul_rn(a[i], p_lo);
-    h[i] = __fmul_rn(a[i], p_hi);
+  for (int i = 0; i < 16; i += 2) {
+    const float2 ai = make_float2(a[i], a[i + 1]);
+    const float2 vl = __fmul2_rn(ai, plo2), vh = __fmul2_rn(ai, phi2);
+    l[i] = vl.x; l[i + 1] = vl.y;
+    h[i] = vh.x; h[i + 1] = vh.y;
   }
-  const uint32_t lo0 = e2m1x8(l[0], l[1], l[2], l[3], l[4], l[5], l[6], l[7]);
-  const uint32_t lo1 = e2m1x8(l[8], l[9], l[10], l[11], l[12], l[13], l[14], l[15]);
-  const uint32_t hi0 = e2m1x8(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]);
-  const uint32_t hi1 = e2m1x8(h[8], h[9], h[10], h[11], h[12], h[13], h[14], h[15]);
-  c0 = lo0;
-  c1 = lo1;
-  if ((lo0 != hi0) | (lo1 != hi1)) {
-    // a quotient sits within the bracket of a rounding boundary: take it exactly
-    const float d = __fmul_rn(e4m3_to_f32(sb), k.s_t);
-    float y[16];
+  lo[0] = e2m1x8(l[0], l[1], l[2], l[3], l[4], l[5], l[6], l[7]);
+  lo[1] = e2m1x8(l[8], l[9], l[10], l[11], l[12], l[13], l[14], l[15]);
+  hi[0] = e2m1x8(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]);
+  hi[1] = e2m1x8(h[8], h[9], h[10], h[11], h[12], h[13], h[14], h[15]);
+}
+
+// |x| of element i (0..7) of a unit, selected without indexing the register
+// array dynamically (which would move it to local memory).
+template <typename InT>
+__device__ __forceinline__ float elem_abs(const Raw<InT>& r, uint32_t i);
+template <>
+__device__ __forceinline__ float elem_abs<__nv_bfloat16>(const Raw<__nv_bfloat16>& r, uint32_t i) {
+  const uint32_t j = i >> 1;
+  uint32_t w = r.w[0];
+  w = j == 1 ? r.w[1] : w;
+  w = j == 2 ? r.w[2] : w;
+  w = j == 3 ? r.w[3] : w;
+  w &= 0x7FFF7FFFu;
+  return __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+}
+template <>
+__device__ __forceinline__ float elem_abs<float>(const Raw<float>& r, uint32_t i) {
+  uint32_t w = r.w[0];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(a[i], d);
-    c0 = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-    c1 = e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+  for (uint32_t j = 1; j < 8; ++j) w = i == j ? r.w[j] : w;
+  return __uint_as_float(w & 0x7FFFFFFFu);
+}
+
+// Replace the codes of a unit whose two bracket codes differ (nonzero nibbles
+// of diff) by the codes of the IEEE quotients |x| / d, d = RN(s_b s_t).
+template <typename InT>
+__device__ __forceinline__ uint32_t patch_codes(const Raw<InT>& r, uint32_t c, uint32_t diff,
+                                                float d) {
+  while (diff) {
+    const uint32_t sh = (__ffs(diff) - 1) & ~3u;
+    c = (c & ~(0xFu << sh)) | (e2m1_of_quotient(elem_abs<InT>(r, sh >> 2), d) << sh);
+    diff &= ~(0xFu << sh);
   }
+  return c;
 }
 
 __device__ __forceinline__ void fill_inv_table(float* tab) {
@@ -238,26 +285,37 @@ __device__ __forceinline__ void fill_inv_table(float* tab) {
     tab[b] = (b == 0 || b == 0x7F) ? 0.0f : __frcp_rn(e4m3_to_f32(b));
 }
 
-// Resolve the tensor scale of plane `plane`: from s_t_in, or amax / 2688.
-__device__ __forceinline__ float plane_scale(const float* s_t_in, const uint32_t* ws, int plane) {
+// Thread 0 of every CTA calls this once.  It returns the plane's tensor scale:
+// s_t_in if given, else amax / 2688 with the amax the producer accumulated
+// (amax_in) or the one this call's amax pass left in the workspace.  An amax
+// word is read once per CTA; the CTA then checks in on the plane's counter
+// (release: the read is ordered before the check-in) and the CTA that checks
+// in last (acquire: every other read happened before) zeroes the amax word and
+// the counter for the next call.  Checking in right after the read keeps the
+// wait for the atomic off the CTA's exit.
+__device__ __forceinline__ float take_scale(const float* s_t_in, float* amax_in, uint32_t* ws,
+                                            int plane) {
   if (s_t_in) return *s_t_in;
-  float amax = __uint_as_float(ws[kWsAmax0 / 4 + plane]);
-  return __fdiv_rn(amax, 2688.0f);
+  uint32_t* const word = amax_in ? reinterpret_cast<uint32_t*>(amax_in) : ws + kWsAmax0 / 4 + plane;
+  uint32_t* const counter = ws + kWsCount0 / 4 + plane;
+  uint32_t bits, done;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(bits) : "l"(word) : "memory");
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+               : "=r"(done)
+               : "l"(counter)
+               : "memory");
+  if (done == gridDim.x - 1) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(word) : "memory");
+    asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(counter) : "memory");
+  }
+  return __fdiv_rn(__uint_as_float(bits), 2688.0f);
 }
 
-// The last CTA of a plane to finish clears that plane's amax and counter,
-// after every CTA of the plane has read the amax.
-__device__ __forceinline__ void self_clean(uint32_t* ws, int plane) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    uint32_t done = atomicAdd(ws + kWsCount0 / 4 + plane, 1u);
-    if (done == gridDim.x - 1) {
-      atomicExch(ws + kWsAmax0 / 4 + plane, 0u);
-      atomicExch(ws + kWsCount0 / 4 + plane, 0u);
-    }
-  }
-}
+// Input blocks a thread keeps in flight while it encodes the ones it holds.
+template <typename InT>
+struct Prefetch {
+  static constexpr int kDepth = 1;
+};
 
 // ---- dense tensors
 struct QuantArgs {
@@ -266,6 +324,7 @@ struct QuantArgs {
   uint8_t* sf;
   float* s_t_out;
   const float* s_t_in;
+  float* amax_in;
   uint32_t* ws;
   uint32_t nkb;          // blocks per row
   FastDiv nkb_div;
@@ -284,22 +343,45 @@ __device__ __forceinline__ uint32_t sf_mma_offset(uint32_t row, uint32_t kb, uin
 template <typename InT>
 __device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, const float* inv_tab,
                                                    const ScaleConsts& k, uint2& codes) {
-  float a[16];
-  uint32_t s0, s1;
-  const uint32_t mx = max(unpack_unit<InT>(raw.h[0], a, s0), unpack_unit<InT>(raw.h[1], a + 8, s1));
-  const uint32_t sb = block_scale(__uint_as_float(mx), k);
-  uint32_t c0, c1;
-  encode_block(a, sb, inv_tab[sb & 0x7Fu], k, c0, c1);
-  codes = sb ? make_uint2(c0 | s0, c1 | s1) : make_uint2(0u, 0u);
+  uint32_t s0, s1, sb, lo[2], hi[2];
+  {
+    float a[16];
+    const uint32_t mx =
+        max(unpack_unit<InT>(raw.h[0], a, s0), unpack_unit<InT>(raw.h[1], a + 8, s1));
+    sb = block_scale(__uint_as_float(mx), k);
+    bracket_codes(a, inv_tab[sb & 0x7Fu], k, lo, hi);
+  }
+  const uint32_t diff0 = lo[0] ^ hi[0], diff1 = lo[1] ^ hi[1];
+  if (diff0 | diff1) {
+    const float d = __fmul_rn(e4m3_to_f32(sb), k.s_t);
+    lo[0] = patch_codes<InT>(raw.h[0], lo[0], diff0, d);
+    lo[1] = patch_codes<InT>(raw.h[1], lo[1], diff1, d);
+  }
+  codes = sb ? make_uint2(lo[0] | s0, lo[1] | s1) : make_uint2(0u, 0u);
   return sb;
 }
 
+// The dense quantizer.  Each thread encodes whole blocks (grid-stride over
+// the tensor's blocks), loading the blocks of its next pass before it encodes
+// the ones it holds; the first loads go out before the tensor scale is known.
 template <typename InT, bool kContig, int kSfLayout>
-__global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs args) {
+__global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args) {
+  constexpr int D = Prefetch<InT>::kDepth;
   __shared__ float inv_tab[128];
+  __shared__ float s_t_shared;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint32_t blocks = args.in.units >> 1;
+  uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x;
+  RawBlock<InT> cur[D];
+#pragma unroll
+  for (int i = 0; i < D; ++i) {
+    const uint32_t b = b0 + i * stride;
+    load_block<InT>(block_ptr<InT, kContig>(args.in, min(b, blocks - 1)), cur[i]);
+  }
+  if (threadIdx.x == 0) s_t_shared = take_scale(args.s_t_in, args.amax_in, args.ws, 0);
   fill_inv_table(inv_tab);
   __syncthreads();
-  const float s_t = plane_scale(args.s_t_in, args.ws, 0);
+  const float s_t = s_t_shared;
   const bool in_domain = tensor_scale_in_domain(s_t);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     *args.s_t_out = s_t;
@@ -307,30 +389,28 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs args) {
   }
   if (in_domain) {
     const ScaleConsts k = make_consts(s_t);
-    const uint32_t stride = gridDim.x * blockDim.x;
-    const uint32_t blocks = args.in.units >> 1;
-    for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < blocks;
-         b0 += kUnroll * stride) {
-      RawBlock<InT> raw[kUnroll];
+    for (; b0 < blocks; b0 += D * stride) {
+      RawBlock<InT> nxt[D];
 #pragma unroll
-      for (int i = 0; i < kUnroll; ++i) {
-        const uint32_t b = b0 + i * stride;
-        const bool valid = b < blocks;
-        load_block<InT>(valid ? block_ptr<InT, kContig>(args.in, b) : nullptr, valid, raw[i]);
+      for (int i = 0; i < D; ++i) {
+        const uint32_t b = b0 + (D + i) * stride;
+        load_block<InT>(block_ptr<InT, kContig>(args.in, min(b, blocks - 1)), nxt[i]);
       }
 #pragma unroll
-      for (int i = 0; i < kUnroll; ++i) {
+      for (int i = 0; i < D; ++i) {
         const uint32_t b = b0 + i * stride;
-        if (b >= blocks) break;
-        uint2 codes;
-        const uint32_t sb = quantize_block<InT>(raw[i], inv_tab, k, codes);
-        reinterpret_cast<uint2*>(args.codes)[b] = codes;
-        if (kSfLayout == NVFP4_SF_ROWMAJOR) {
-          args.sf[b] = uint8_t(sb);
-        } else {
-          const uint32_t row = fast_div(args.nkb_div, b);
-          args.sf[sf_mma_offset(row, b - row * args.nkb, args.ktiles)] = uint8_t(sb);
+        if (b < blocks) {
+          uint2 codes;
+          const uint32_t sb = quantize_block<InT>(cur[i], inv_tab, k, codes);
+          reinterpret_cast<uint2*>(args.codes)[b] = codes;
+          if (kSfLayout == NVFP4_SF_ROWMAJOR) {
+            args.sf[b] = uint8_t(sb);
+          } else {
+            const uint32_t row = fast_div(args.nkb_div, b);
+            args.sf[sf_mma_offset(row, b - row * args.nkb, args.ktiles)] = uint8_t(sb);
+          }
         }
+        cur[i] = nxt[i];
       }
     }
   }
@@ -354,7 +434,6 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs args) {
       args.sf[sf_mma_offset(row, kb, args.ktiles)] = 0;
     }
   }
-  if (!args.s_t_in) self_clean(args.ws, 0);
 }
 
 // ---- KV-cache chunks (K and V planes in one launch, blockIdx.y)
@@ -371,59 +450,104 @@ struct KvQuantArgs {
 };
 
 template <bool kContig>
-__global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(KvQuantArgs args) {
+__global__ void __launch_bounds__(kQuantThreads, 4) kv_quant_kernel(KvQuantArgs args) {
+  constexpr int D = Prefetch<__nv_bfloat16>::kDepth;
   __shared__ float inv_tab[128];
+  __shared__ float s_t_shared;
+  const int plane = blockIdx.y;
+  const InMap m = plane == 0 ? args.in[0] : args.in[1];
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint32_t blocks = m.units >> 1;
+  uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x;
+  RawBlock<__nv_bfloat16> cur[D];
+#pragma unroll
+  for (int i = 0; i < D; ++i) {
+    const uint32_t b = b0 + i * stride;
+    load_block<__nv_bfloat16>(block_ptr<__nv_bfloat16, kContig>(m, min(b, blocks - 1)),
+                              cur[i]);
+  }
+  if (threadIdx.x == 0) s_t_shared = take_scale(nullptr, nullptr, args.ws, plane);
   fill_inv_table(inv_tab);
   __syncthreads();
-  const int plane = blockIdx.y;
-  const float s_t = plane_scale(nullptr, args.ws, plane);
+  const float s_t = s_t_shared;
   const bool in_domain = tensor_scale_in_domain(s_t);
   if (blockIdx.x == 0 && threadIdx.x < args.n_frames)
     args.st[plane][args.slots[threadIdx.x]] = s_t;
   if (blockIdx.x == 0 && threadIdx.x == 0 && !in_domain)
     record_status(args.ws + kWsStatus / 4, NVFP4_ERR_DOMAIN);
   if (in_domain) {
-    const InMap m = plane == 0 ? args.in[0] : args.in[1];
     uint8_t* const codes_pool = plane == 0 ? args.codes[0] : args.codes[1];
     uint8_t* const sf_pool = plane == 0 ? args.sf[0] : args.sf[1];
     const ScaleConsts k = make_consts(s_t);
-    const uint32_t stride = gridDim.x * blockDim.x;
-    const uint32_t blocks = m.units >> 1;
     const uint32_t bpf = args.units_per_frame >> 1;  // blocks per frame
-    for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < blocks;
-         b0 += kUnroll * stride) {
-      RawBlock<__nv_bfloat16> raw[kUnroll];
+    for (; b0 < blocks; b0 += D * stride) {
+      RawBlock<__nv_bfloat16> nxt[D];
 #pragma unroll
-      for (int i = 0; i < kUnroll; ++i) {
-        const uint32_t b = b0 + i * stride;
-        const bool valid = b < blocks;
-        load_block<__nv_bfloat16>(valid ? block_ptr<__nv_bfloat16, kContig>(m, b) : nullptr,
-                                  valid, raw[i]);
+      for (int i = 0; i < D; ++i) {
+        const uint32_t b = b0 + (D + i) * stride;
+        load_block<__nv_bfloat16>(block_ptr<__nv_bfloat16, kContig>(m, min(b, blocks - 1)),
+                                  nxt[i]);
       }
 #pragma unroll
-      for (int i = 0; i < kUnroll; ++i) {
+      for (int i = 0; i < D; ++i) {
         const uint32_t b = b0 + i * stride;
-        if (b >= blocks) break;
-        uint2 codes;
-        const uint32_t sb = quantize_block<__nv_bfloat16>(raw[i], inv_tab, k, codes);
-        const uint32_t f = fast_div(args.bpf_div, b);
-        const uint32_t bf = b - f * bpf;
-        const size_t slot = size_t(args.slots[f]);
-        reinterpret_cast<uint2*>(codes_pool + slot * bpf * 8)[bf] = codes;
-        sf_pool[slot * bpf + bf] = uint8_t(sb);
+        if (b < blocks) {
+          uint2 codes;
+          const uint32_t sb = quantize_block<__nv_bfloat16>(cur[i], inv_tab, k, codes);
+          const uint32_t f = fast_div(args.bpf_div, b);
+          const uint32_t bf = b - f * bpf;
+          const size_t slot = size_t(args.slots[f]);
+          reinterpret_cast<uint2*>(codes_pool + slot * bpf * 8)[bf] = codes;
+          sf_pool[slot * bpf + bf] = uint8_t(sb);
+        }
+        cur[i] = nxt[i];
       }
     }
   }
-  self_clean(args.ws, plane);
 }
 
 // ---------------------------------------------------------------- launchers
-static int grid_for(uint32_t units, int sm_count) {
+// CTAs of `kernel` resident on one SM at once.
+template <typename Kernel>
+static int resident_per_sm(Kernel kernel) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kQuantThreads, 0) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  return n;
+}
+
+// CTAs per plane: enough for `per_thread` blocks per thread, at most one
+// resident wave of the whole launch (all `planes` planes) so that no CTA
+// waits for another to leave.
+static int wave_grid(uint32_t units, uint32_t per_thread, int per_sm, int sm_count, int planes) {
   const uint64_t blocks = uint64_t(units) / 2;
-  uint64_t want = (blocks + kQuantThreads * kUnroll - 1) / (kQuantThreads * kUnroll);
-  uint64_t cap = uint64_t(sm_count) * 8;
+  uint64_t want = (blocks + kQuantThreads * per_thread - 1) / (kQuantThreads * per_thread);
+  uint64_t cap = uint64_t(per_sm) * uint64_t(sm_count) / uint64_t(planes);
+  if (cap < 1) cap = 1;
   if (want < 1) want = 1;
   return int(want < cap ? want : cap);
+}
+
+template <typename InT, bool kContig>
+static void launch_amax(const AmaxArgs& aa, int planes, int sm_count, cudaStream_t st) {
+  static const int per_sm = resident_per_sm(amax_kernel<InT, kContig>);
+  const int grid = wave_grid(aa.in[0].units, 2, per_sm, sm_count, planes);
+  amax_kernel<InT, kContig><<<dim3(grid, planes), kQuantThreads, 0, st>>>(aa);
+}
+
+template <typename InT, bool kContig, int kSfLayout>
+static void launch_encode(const QuantArgs& a, int sm_count, cudaStream_t st) {
+  static const int per_sm = resident_per_sm(quant_kernel<InT, kContig, kSfLayout>);
+  const int grid = wave_grid(a.in.units, 1, per_sm, sm_count, 1);
+  quant_kernel<InT, kContig, kSfLayout><<<grid, kQuantThreads, 0, st>>>(a);
+}
+
+template <bool kContig>
+static void launch_kv_encode(const KvQuantArgs& a, int sm_count, cudaStream_t st) {
+  static const int per_sm = resident_per_sm(kv_quant_kernel<kContig>);
+  const int grid = wave_grid(a.in[0].units, 1, per_sm, sm_count, 2);
+  kv_quant_kernel<kContig><<<dim3(grid, 2), kQuantThreads, 0, st>>>(a);
 }
 
 static InMap make_inmap(const void* x, int64_t rows_total, int64_t cols, int64_t rows_per_group,
@@ -442,16 +566,15 @@ template <typename InT>
 static cudaError_t launch_quant_t(const LaunchQuant& q, cudaStream_t st) {
   const bool contig = (q.ld == q.cols);
   InMap m = make_inmap(q.x, q.rows, q.cols, 1, q.ld, 0);
-  const int grid = grid_for(m.units, q.sm_count);
-  if (!q.s_t_in) {
+  if (!q.s_t_in && !q.amax_in) {
     AmaxArgs aa;
     aa.in[0] = m;
     aa.in[1] = m;
     aa.ws = static_cast<uint32_t*>(q.ws);
     if (contig)
-      amax_kernel<InT, true><<<dim3(grid, 1), kQuantThreads, 0, st>>>(aa);
+      launch_amax<InT, true>(aa, 1, q.sm_count, st);
     else
-      amax_kernel<InT, false><<<dim3(grid, 1), kQuantThreads, 0, st>>>(aa);
+      launch_amax<InT, false>(aa, 1, q.sm_count, st);
   }
   QuantArgs a;
   a.in = m;
@@ -459,6 +582,7 @@ static cudaError_t launch_quant_t(const LaunchQuant& q, cudaStream_t st) {
   a.sf = q.sf;
   a.s_t_out = q.s_t_out;
   a.s_t_in = q.s_t_in;
+  a.amax_in = q.amax_in;
   a.ws = static_cast<uint32_t*>(q.ws);
   a.nkb = uint32_t(q.cols / 16);
   a.nkb_div = make_fastdiv(a.nkb);
@@ -467,11 +591,11 @@ static cudaError_t launch_quant_t(const LaunchQuant& q, cudaStream_t st) {
   a.rows_pad = uint32_t((q.rows + 127) / 128 * 128);
   const bool mma = q.sf_layout == NVFP4_SF_MMA128x4;
   if (contig) {
-    if (mma) quant_kernel<InT, true, NVFP4_SF_MMA128x4><<<grid, kQuantThreads, 0, st>>>(a);
-    else quant_kernel<InT, true, NVFP4_SF_ROWMAJOR><<<grid, kQuantThreads, 0, st>>>(a);
+    if (mma) launch_encode<InT, true, NVFP4_SF_MMA128x4>(a, q.sm_count, st);
+    else launch_encode<InT, true, NVFP4_SF_ROWMAJOR>(a, q.sm_count, st);
   } else {
-    if (mma) quant_kernel<InT, false, NVFP4_SF_MMA128x4><<<grid, kQuantThreads, 0, st>>>(a);
-    else quant_kernel<InT, false, NVFP4_SF_ROWMAJOR><<<grid, kQuantThreads, 0, st>>>(a);
+    if (mma) launch_encode<InT, false, NVFP4_SF_MMA128x4>(a, q.sm_count, st);
+    else launch_encode<InT, false, NVFP4_SF_ROWMAJOR>(a, q.sm_count, st);
   }
   return cudaGetLastError();
 }
@@ -502,13 +626,12 @@ cudaError_t launch_kv_quant(const LaunchKvQuant& q, cudaStream_t st) {
   ka.bpf_div = make_fastdiv(ka.units_per_frame / 2);
   for (int f = 0; f < NVFP4_KV_MAX_CHUNK_FRAMES; ++f) ka.slots[f] = f < q.n_frames ? q.slots[f] : 0;
   ka.n_frames = q.n_frames;
-  const int grid = grid_for(aa.in[0].units, q.sm_count);
   if (contig) {
-    amax_kernel<__nv_bfloat16, true><<<dim3(grid, 2), kQuantThreads, 0, st>>>(aa);
-    kv_quant_kernel<true><<<dim3(grid, 2), kQuantThreads, 0, st>>>(ka);
+    launch_amax<__nv_bfloat16, true>(aa, 2, q.sm_count, st);
+    launch_kv_encode<true>(ka, q.sm_count, st);
   } else {
-    amax_kernel<__nv_bfloat16, false><<<dim3(grid, 2), kQuantThreads, 0, st>>>(aa);
-    kv_quant_kernel<false><<<dim3(grid, 2), kQuantThreads, 0, st>>>(ka);
+    launch_amax<__nv_bfloat16, false>(aa, 2, q.sm_count, st);
+    launch_kv_encode<false>(ka, q.sm_count, st);
   }
   return cudaGetLastError();
 }

@@ -87,8 +87,15 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def quantize(x: torch.Tensor, sf_layout: int = N.SF_MMA128x4, s_t: Optional[torch.Tensor] = None,
-             out: Optional[NVFP4Tensor] = None, ws: Optional[torch.Tensor] = None) -> NVFP4Tensor:
-    """nvfp4_quantize: x is a 2-D bf16/fp32 CUDA tensor with unit column stride."""
+             out: Optional[NVFP4Tensor] = None, ws: Optional[torch.Tensor] = None,
+             amax_in: Optional[torch.Tensor] = None) -> NVFP4Tensor:
+    """nvfp4_quantize: x is a 2-D bf16/fp32 CUDA tensor with unit column stride.
+
+    s_t:     a one-element fp32 tensor holding the tensor scale to use, or None.
+    amax_in: a one-element fp32 tensor holding max|x| as accumulated by the
+             producer (``gemm(..., c_amax=)``); the amax pass is skipped and the
+             word is reset to 0 when the launch ends.  Exclusive with s_t.
+    """
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("quantize expects a 2-D tensor with contiguous rows")
     rows, cols = x.shape
@@ -97,8 +104,8 @@ def quantize(x: torch.Tensor, sf_layout: int = N.SF_MMA128x4, s_t: Optional[torc
     ws = workspace(x.device) if ws is None else ws
     st = out.c_struct()
     N.check(N.lib().nvfp4_quantize(x.data_ptr(), _dtype_code(x), rows, cols, x.stride(0),
-                                   ctypes.byref(st), _ptr(s_t), ws.data_ptr(), ws.numel(),
-                                   _stream()), "nvfp4_quantize")
+                                   ctypes.byref(st), _ptr(s_t), _ptr(amax_in), ws.data_ptr(),
+                                   ws.numel(), _stream()), "nvfp4_quantize")
     return out
 
 
@@ -113,15 +120,20 @@ def dequantize(t: NVFP4Tensor, out: Optional[torch.Tensor] = None) -> torch.Tens
 
 
 def gemm(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype: torch.dtype = torch.bfloat16,
-         out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """nvfp4_gemm: C = A W^T, [a.rows, w.rows] in bf16 or fp32."""
+         out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+         c_amax: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """nvfp4_gemm: C = A W^T, [a.rows, w.rows] in bf16 or fp32.
+
+    c_amax: a one-element fp32 tensor that starts at 0 (or at a smaller running
+            max); the kernel raises it to max|C| over the values it stores.
+    """
     if out is None:
         out = torch.empty(a.rows, w.rows, dtype=out_dtype, device=a.device)
     ws = workspace(a.device) if ws is None else ws
     sa, sw = a.c_struct(), w.c_struct()
     N.check(N.lib().nvfp4_gemm(ctypes.byref(sa), ctypes.byref(sw), out.data_ptr(),
-                               _dtype_code(out), out.stride(0), ws.data_ptr(), ws.numel(),
-                               _stream()), "nvfp4_gemm")
+                               _dtype_code(out), out.stride(0), _ptr(c_amax), ws.data_ptr(),
+                               ws.numel(), _stream()), "nvfp4_gemm")
     return out
 
 

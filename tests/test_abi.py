@@ -56,25 +56,32 @@ def test_quantize_rejects(L):
     t = _tensor()
     ws = FAKE
     q = L.nvfp4_quantize
-    assert q(None, N.BF16, 256, 256, 256, ctypes.byref(t), None, ws, 256, None) == N.ERR_INVALID_ARG
-    assert q(FAKE, 9, 256, 256, 256, ctypes.byref(t), None, ws, 256, None) == N.ERR_INVALID_ARG
-    bad = _tensor(cols=40)
-    assert q(FAKE, N.BF16, 256, 40, 40, ctypes.byref(bad), None, ws, 256,
-             None) == N.ERR_UNSUPPORTED_SHAPE
-    assert q(FAKE, N.BF16, 255, 256, 256, ctypes.byref(t), None, ws, 256,
-             None) == N.ERR_INVALID_ARG  # rows differ from out->rows
-    assert q(FAKE + 2, N.BF16, 256, 256, 256, ctypes.byref(t), None, ws, 256,
+    assert q(None, N.BF16, 256, 256, 256, ctypes.byref(t), None, None, ws, 256,
+             None) == N.ERR_INVALID_ARG
+    assert q(FAKE, 9, 256, 256, 256, ctypes.byref(t), None, None, ws, 256,
+             None) == N.ERR_INVALID_ARG
+    # a given tensor scale and a producer amax are exclusive
+    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), FAKE, FAKE, ws, 256,
+             None) == N.ERR_INVALID_ARG
+    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, FAKE + 2, ws, 256,
              None) == N.ERR_MISALIGNED
-    assert q(FAKE, N.BF16, 256, 256, 260, ctypes.byref(t), None, ws, 256,
+    bad = _tensor(cols=40)
+    assert q(FAKE, N.BF16, 256, 40, 40, ctypes.byref(bad), None, None, ws, 256,
+             None) == N.ERR_UNSUPPORTED_SHAPE
+    assert q(FAKE, N.BF16, 255, 256, 256, ctypes.byref(t), None, None, ws, 256,
+             None) == N.ERR_INVALID_ARG  # rows differ from out->rows
+    assert q(FAKE + 2, N.BF16, 256, 256, 256, ctypes.byref(t), None, None, ws, 256,
+             None) == N.ERR_MISALIGNED
+    assert q(FAKE, N.BF16, 256, 256, 260, ctypes.byref(t), None, None, ws, 256,
              None) == N.ERR_MISALIGNED  # 520-byte row stride
     mis = _tensor(codes=FAKE + 8)
-    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(mis), None, ws, 256,
+    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(mis), None, None, ws, 256,
              None) == N.ERR_MISALIGNED
-    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, ws, 8, None) == N.ERR_WORKSPACE
-    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, None, 256,
+    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, None, ws, 8, None) == N.ERR_WORKSPACE
+    assert q(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, None, None, 256,
              None) == N.ERR_WORKSPACE
     huge = _tensor(rows=1 << 30, cols=256)
-    assert q(FAKE, N.BF16, 1 << 30, 256, 256, ctypes.byref(huge), None, ws, 256,
+    assert q(FAKE, N.BF16, 1 << 30, 256, 256, ctypes.byref(huge), None, None, ws, 256,
              None) == N.ERR_UNSUPPORTED_SHAPE
 
 
@@ -82,7 +89,7 @@ def test_gemm_rejects(L):
     a = _tensor(rows=2640, cols=3072)
     w = _tensor(rows=9216, cols=3072)
     g = L.nvfp4_gemm
-    ok_args = (FAKE, N.BF16, 9216, FAKE, 256, None)
+    ok_args = (FAKE, N.BF16, 9216, None, FAKE, 256, None)
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9216, cols=3072, layout=N.SF_ROWMAJOR)),
              *ok_args) == N.ERR_INVALID_ARG
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9216, cols=2048)),
@@ -90,15 +97,17 @@ def test_gemm_rejects(L):
     assert g(ctypes.byref(_tensor(rows=2640, cols=3056)),
              ctypes.byref(_tensor(rows=9216, cols=3056)), *ok_args) == N.ERR_UNSUPPORTED_SHAPE
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9200, cols=3072)),
-             FAKE, N.BF16, 9216, FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # N % 256
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9000, FAKE, 256,
+             FAKE, N.BF16, 9216, None, FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # N % 256
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9000, None, FAKE, 256,
              None) == N.ERR_INVALID_ARG  # ldc < N
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9220, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9220, None, FAKE, 256,
              None) == N.ERR_MISALIGNED
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, 5, 9216, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, 5, 9216, None, FAKE, 256,
              None) == N.ERR_INVALID_ARG
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, FAKE, 4,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, None, FAKE, 4,
              None) == N.ERR_WORKSPACE
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, FAKE + 1, FAKE, 256,
+             None) == N.ERR_MISALIGNED  # c_amax
 
 
 def _cache(n_slots=12, tpf=880, heads=24, hd=128):
@@ -137,5 +146,5 @@ def test_no_gpu_means_arch_error_not_fallback(L):
     """With every argument valid but no sm_100 device, the call refuses with
     NVFP4_ERR_ARCH instead of computing anything on the host."""
     t = _tensor()
-    assert L.nvfp4_quantize(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, FAKE, 256,
+    assert L.nvfp4_quantize(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, None, FAKE, 256,
                             None) == N.ERR_ARCH

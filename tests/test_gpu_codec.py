@@ -121,6 +121,21 @@ def test_ties_fp32(orc):
         assert_quant_equal(orc, q, x, layout)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_dense_ties_power_of_two_tensor_scale(orc, dtype):
+    """bf16-valued data with amax 5.25, so s_t = 5.25 / 2688 = 2^-9 exactly:
+    many quotients land exactly on E2M1 and E4M3 rounding boundaries, in most
+    warps of the launch (every element position of a block gets some)."""
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(1000, 4096, generator=g) * 1.5).clamp(-5.25, 5.25)
+    x = x.to(torch.bfloat16).to(dtype)
+    x[7, 123] = 5.25
+    for layout in LAYOUTS:
+        q = _q(x, layout)
+        assert float(q.s_t.cpu()[0]) == 2.0 ** -9
+        assert_quant_equal(orc, q, bits(x), layout)
+
+
 def test_zero_and_special_values(orc):
     x = torch.zeros(130, 64)
     q = _q(x, nv.SF_MMA128x4)
