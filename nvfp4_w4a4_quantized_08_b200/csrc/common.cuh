@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t fast_div(const FastDiv& f, uint32_t n) {
 }
 
 // ---------------------------------------------------------------- formats
-// Eight non-negative binary32 values -> eight E2M1 codes packed little-endian
+// Eight binary32 values -> eight E2M1 codes (sign bit 3) packed little-endian
 // (value i in nibble i).  cvt.e2m1x2 puts its first source in the high nibble.
 __device__ __forceinline__ uint32_t e2m1x8(float y0, float y1, float y2, float y3, float y4,
                                            float y5, float y6, float y7) {
@@ -119,6 +119,21 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
   asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
+}
+
+// 32-byte store (sm_100 256-bit access); p must be 32-byte aligned.
+__device__ __forceinline__ void st_v8(void* p, uint4 a, uint4 b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x),
+               "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
+// 32-byte read-only load (sm_100 256-bit access); p must be 32-byte aligned.
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint4& a, uint4& b) {
+  asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z),
+                 "=r"(b.w)
+               : "l"(p));
 }
 
 }  // namespace nvfp4

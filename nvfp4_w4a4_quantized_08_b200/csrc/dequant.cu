@@ -93,10 +93,22 @@ struct DequantArgs {
   uint32_t ktiles;
 };
 
+// Store one decoded block (32 bytes): one 256-bit store when the destination
+// is 32-byte aligned (a warp then writes whole sectors), else two 128-bit ones.
+template <bool kWide>
+__device__ __forceinline__ void store_block(uint8_t* dst, uint4 lo, uint4 hi) {
+  if (kWide) {
+    st_v8(dst, lo, hi);
+  } else {
+    st_v4(dst, lo);
+    st_v4(dst + 16, hi);
+  }
+}
+
 // A thread decodes whole blocks (8 code bytes in, 32 bytes out), kDqUnroll
 // of them per pass with all their loads issued first.  Threads past the end
 // load the last block again and store nothing.
-template <int kSfLayout, bool kContig>
+template <int kSfLayout, bool kContig, bool kWide>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(DequantArgs a) {
   const float s_t = *a.s_t;
   const uint32_t stride = gridDim.x * blockDim.x;
@@ -121,8 +133,7 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(DequantArgs a) {
       const BlockLut l = make_lut(sb[i], s_t);
       uint8_t* dst = kContig ? a.out + 32 * size_t(b)
                              : a.out + 2 * (int64_t(row[i]) * a.ld + 16 * int64_t(kb[i]));
-      st_v4(dst, decode8(l, c[i].x));
-      st_v4(dst + 16, decode8(l, c[i].y));
+      store_block<kWide>(dst, decode8(l, c[i].x), decode8(l, c[i].y));
     }
   }
 }
@@ -138,6 +149,7 @@ struct KvDequantArgs {
   int32_t slots[NVFP4_KV_MAX_WINDOW_SLOTS];
 };
 
+template <bool kWide>
 __global__ void __launch_bounds__(kDqThreads) kv_dequant_kernel(KvDequantArgs a) {
   const int plane = blockIdx.y;
   const uint8_t* codes = plane == 0 ? a.codes[0] : a.codes[1];
@@ -166,8 +178,7 @@ __global__ void __launch_bounds__(kDqThreads) kv_dequant_kernel(KvDequantArgs a)
       const uint32_t b = b0 + i * stride;
       if (b >= a.blocks) break;
       const BlockLut l = make_lut(sb[i], st[i]);
-      st_v4(out + 32 * size_t(b), decode8(l, c[i].x));
-      st_v4(out + 32 * size_t(b) + 16, decode8(l, c[i].y));
+      store_block<kWide>(out + 32 * size_t(b), decode8(l, c[i].x), decode8(l, c[i].y));
     }
   }
 }
@@ -200,15 +211,26 @@ cudaError_t launch_dequantize(const LaunchDequant& d, cudaStream_t st) {
   a.ktiles = (a.nkb + 3) / 4;
   const bool contig = d.ld == d.cols;
   const bool mma = d.sf_layout == NVFP4_SF_MMA128x4;
+  const bool wide = reinterpret_cast<uintptr_t>(d.out) % 32 == 0 && (contig || d.ld % 16 == 0);
   auto launch = [&](auto kernel) {
     kernel<<<dq_grid(kernel, a.blocks, d.sm_count, 1), kDqThreads, 0, st>>>(a);
   };
-  if (mma) {
-    if (contig) launch(dequant_kernel<NVFP4_SF_MMA128x4, true>);
-    else launch(dequant_kernel<NVFP4_SF_MMA128x4, false>);
+  if (wide) {
+    if (mma) {
+      if (contig) launch(dequant_kernel<NVFP4_SF_MMA128x4, true, true>);
+      else launch(dequant_kernel<NVFP4_SF_MMA128x4, false, true>);
+    } else {
+      if (contig) launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true, true>);
+      else launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false, true>);
+    }
   } else {
-    if (contig) launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true>);
-    else launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false>);
+    if (mma) {
+      if (contig) launch(dequant_kernel<NVFP4_SF_MMA128x4, true, false>);
+      else launch(dequant_kernel<NVFP4_SF_MMA128x4, false, false>);
+    } else {
+      if (contig) launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true, false>);
+      else launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false, false>);
+    }
   }
   return cudaGetLastError();
 }
@@ -224,8 +246,15 @@ cudaError_t launch_kv_dequant(const LaunchKvDequant& d, cudaStream_t st) {
   a.bpf_div = make_fastdiv(a.blocks_per_frame);
   a.blocks = uint32_t(int64_t(d.n) * a.blocks_per_frame);
   for (int i = 0; i < NVFP4_KV_MAX_WINDOW_SLOTS; ++i) a.slots[i] = i < d.n ? d.slots[i] : 0;
-  const int grid = dq_grid(kv_dequant_kernel, a.blocks, d.sm_count, 2);
-  kv_dequant_kernel<<<dim3(grid, 2), kDqThreads, 0, st>>>(a);
+  const bool wide = reinterpret_cast<uintptr_t>(d.k_out) % 32 == 0 &&
+                    reinterpret_cast<uintptr_t>(d.v_out) % 32 == 0;
+  if (wide) {
+    const int grid = dq_grid(kv_dequant_kernel<true>, a.blocks, d.sm_count, 2);
+    kv_dequant_kernel<true><<<dim3(grid, 2), kDqThreads, 0, st>>>(a);
+  } else {
+    const int grid = dq_grid(kv_dequant_kernel<false>, a.blocks, d.sm_count, 2);
+    kv_dequant_kernel<false><<<dim3(grid, 2), kDqThreads, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 

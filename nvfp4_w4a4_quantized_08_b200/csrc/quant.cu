@@ -80,44 +80,41 @@ __device__ __forceinline__ void load_unit<float>(const float* p, Raw<float>& r) 
   r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
 }
 
-// |x| of the 8 elements as binary32, their max (as binary32 bits; NaN/Inf
-// inputs give bits >= 0x7F800000) and the sign bits placed at bit 3 of each
-// output nibble.
+// max |x| of the 8 elements of a unit, as binary32 bits (NaN and Inf inputs
+// give bits >= 0x7F800000, so they dominate the max).
 template <typename InT>
-__device__ __forceinline__ uint32_t unpack_unit(const Raw<InT>& r, float a[8], uint32_t& signs);
+__device__ __forceinline__ uint32_t unit_absmax(const Raw<InT>& r);
 template <>
-__device__ __forceinline__ uint32_t unpack_unit<__nv_bfloat16>(const Raw<__nv_bfloat16>& r,
-                                                               float a[8], uint32_t& signs) {
-  uint32_t m[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    m[j] = r.w[j] & 0x7FFF7FFFu;
-    a[2 * j] = __uint_as_float(m[j] << 16);
-    a[2 * j + 1] = __uint_as_float(m[j] & 0xFFFF0000u);
-  }
-  uint32_t mx = __vmaxu2(__vmaxu2(m[0], m[1]), __vmaxu2(m[2], m[3]));
-  mx = max(mx & 0xFFFFu, mx >> 16) << 16;
-  // high bytes of the even elements (low halves) and of the odd elements
-  uint32_t p01 = prmt(r.w[0], r.w[1], 0x7351);  // [w0.b1, w1.b1, w0.b3, w1.b3]
-  uint32_t p23 = prmt(r.w[2], r.w[3], 0x7351);
-  uint32_t even = prmt(p01, p23, 0x5410);  // sign of element 2j at bit 8j+7
-  uint32_t odd = prmt(p01, p23, 0x7632);   // sign of element 2j+1 at bit 8j+7
-  signs = ((even >> 4) & 0x08080808u) | (odd & 0x80808080u);
-  return mx;
+__device__ __forceinline__ uint32_t unit_absmax<__nv_bfloat16>(const Raw<__nv_bfloat16>& r) {
+  const uint32_t m = __vmaxu2(__vmaxu2(r.w[0] & 0x7FFF7FFFu, r.w[1] & 0x7FFF7FFFu),
+                              __vmaxu2(r.w[2] & 0x7FFF7FFFu, r.w[3] & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16) << 16;
 }
 template <>
-__device__ __forceinline__ uint32_t unpack_unit<float>(const Raw<float>& r, float a[8],
-                                                       uint32_t& signs) {
+__device__ __forceinline__ uint32_t unit_absmax<float>(const Raw<float>& r) {
   uint32_t mx = 0;
-  signs = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint32_t b = r.w[i] & 0x7FFFFFFFu;
-    a[i] = __uint_as_float(b);
-    mx = max(mx, b);
-    signs |= (r.w[i] >> 31) << (4 * i + 3);
-  }
+  for (int i = 0; i < 8; ++i) mx = max(mx, r.w[i] & 0x7FFFFFFFu);
   return mx;
+}
+
+// The 8 elements of a unit as binary32, sign included (bf16 -> binary32 is
+// exact: the bf16 bits are the high half).
+template <typename InT>
+__device__ __forceinline__ void unit_values(const Raw<InT>& r, float a[8]);
+template <>
+__device__ __forceinline__ void unit_values<__nv_bfloat16>(const Raw<__nv_bfloat16>& r,
+                                                           float a[8]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    a[2 * j] = __uint_as_float(r.w[j] << 16);
+    a[2 * j + 1] = __uint_as_float(r.w[j] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void unit_values<float>(const Raw<float>& r, float a[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(r.w[i]);
 }
 
 // ---------------------------------------------------------------- block access
@@ -161,12 +158,8 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(AmaxArgs args) {
       load_block<InT>(block_ptr<InT, kContig>(m, min(b, blocks - 1)), raw[i]);
     }
 #pragma unroll
-    for (int i = 0; i < kAmaxUnroll; ++i) {
-      float a[8];
-      uint32_t signs;
-      mx = max(mx, unpack_unit<InT>(raw[i].h[0], a, signs));
-      mx = max(mx, unpack_unit<InT>(raw[i].h[1], a, signs));
-    }
+    for (int i = 0; i < kAmaxUnroll; ++i)
+      mx = max(mx, max(unit_absmax<InT>(raw[i].h[0]), unit_absmax<InT>(raw[i].h[1])));
   }
   mx = __reduce_max_sync(0xFFFFFFFFu, mx);
   __shared__ uint32_t warp_max[kQuantThreads / 32];
@@ -220,9 +213,11 @@ __device__ __forceinline__ uint32_t block_scale(float amax_b, const ScaleConsts&
   return k.zero ? 0u : sb;
 }
 
-// Magnitude codes of the 16 elements of a block (|x| in a) for block scale
-// byte sb from the two bracketing products: lo/hi code words of each half.
-// Nibbles where lo and hi differ need the exact quotient.
+// E2M1 codes of the 16 elements of a block (x in a) for block scale byte sb,
+// from the two bracketing products: lo/hi code words of each half.  The codes
+// carry the sign (E2M1 is sign-magnitude and rounding to nearest even is
+// symmetric, so code(-y) = 8 | code(y); a negative value that rounds to zero
+// gives -0).  Nibbles where lo and hi differ need the exact quotient.
 __device__ __forceinline__ void bracket_codes(const float a[16], float inv_sb,
                                               const ScaleConsts& k, uint32_t lo[2],
                                               uint32_t hi[2]) {
@@ -245,36 +240,36 @@ __device__ __forceinline__ void bracket_codes(const float a[16], float inv_sb,
   hi[1] = e2m1x8(h[8], h[9], h[10], h[11], h[12], h[13], h[14], h[15]);
 }
 
-// |x| of element i (0..7) of a unit, selected without indexing the register
-// array dynamically (which would move it to local memory).
+// Element i (0..7) of a unit as binary32, selected without indexing the
+// register array dynamically (which would move it to local memory).
 template <typename InT>
-__device__ __forceinline__ float elem_abs(const Raw<InT>& r, uint32_t i);
+__device__ __forceinline__ float elem_value(const Raw<InT>& r, uint32_t i);
 template <>
-__device__ __forceinline__ float elem_abs<__nv_bfloat16>(const Raw<__nv_bfloat16>& r, uint32_t i) {
+__device__ __forceinline__ float elem_value<__nv_bfloat16>(const Raw<__nv_bfloat16>& r,
+                                                           uint32_t i) {
   const uint32_t j = i >> 1;
   uint32_t w = r.w[0];
   w = j == 1 ? r.w[1] : w;
   w = j == 2 ? r.w[2] : w;
   w = j == 3 ? r.w[3] : w;
-  w &= 0x7FFF7FFFu;
   return __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
 }
 template <>
-__device__ __forceinline__ float elem_abs<float>(const Raw<float>& r, uint32_t i) {
+__device__ __forceinline__ float elem_value<float>(const Raw<float>& r, uint32_t i) {
   uint32_t w = r.w[0];
 #pragma unroll
   for (uint32_t j = 1; j < 8; ++j) w = i == j ? r.w[j] : w;
-  return __uint_as_float(w & 0x7FFFFFFFu);
+  return __uint_as_float(w);
 }
 
 // Replace the codes of a unit whose two bracket codes differ (nonzero nibbles
-// of diff) by the codes of the IEEE quotients |x| / d, d = RN(s_b s_t).
+// of diff) by the codes of the IEEE quotients x / d, d = RN(s_b s_t).
 template <typename InT>
 __device__ __forceinline__ uint32_t patch_codes(const Raw<InT>& r, uint32_t c, uint32_t diff,
                                                 float d) {
   while (diff) {
     const uint32_t sh = (__ffs(diff) - 1) & ~3u;
-    c = (c & ~(0xFu << sh)) | (e2m1_of_quotient(elem_abs<InT>(r, sh >> 2), d) << sh);
+    c = (c & ~(0xFu << sh)) | (e2m1_of_quotient(elem_value<InT>(r, sh >> 2), d) << sh);
     diff &= ~(0xFu << sh);
   }
   return c;
@@ -339,16 +334,17 @@ __device__ __forceinline__ uint32_t sf_mma_offset(uint32_t row, uint32_t kb, uin
 }
 
 // Quantize one block held in `raw`: returns its scale byte and writes its two
-// code words (sign bits included; all +0 when the scale is 0).
+// code words (all +0 when the scale is 0).
 template <typename InT>
 __device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, const float* inv_tab,
                                                    const ScaleConsts& k, uint2& codes) {
-  uint32_t s0, s1, sb, lo[2], hi[2];
+  uint32_t sb, lo[2], hi[2];
   {
-    float a[16];
-    const uint32_t mx =
-        max(unpack_unit<InT>(raw.h[0], a, s0), unpack_unit<InT>(raw.h[1], a + 8, s1));
+    const uint32_t mx = max(unit_absmax<InT>(raw.h[0]), unit_absmax<InT>(raw.h[1]));
     sb = block_scale(__uint_as_float(mx), k);
+    float a[16];
+    unit_values<InT>(raw.h[0], a);
+    unit_values<InT>(raw.h[1], a + 8);
     bracket_codes(a, inv_tab[sb & 0x7Fu], k, lo, hi);
   }
   const uint32_t diff0 = lo[0] ^ hi[0], diff1 = lo[1] ^ hi[1];
@@ -357,7 +353,7 @@ __device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, con
     lo[0] = patch_codes<InT>(raw.h[0], lo[0], diff0, d);
     lo[1] = patch_codes<InT>(raw.h[1], lo[1], diff1, d);
   }
-  codes = sb ? make_uint2(lo[0] | s0, lo[1] | s1) : make_uint2(0u, 0u);
+  codes = sb ? make_uint2(lo[0], lo[1]) : make_uint2(0u, 0u);
   return sb;
 }
 

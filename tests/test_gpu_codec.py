@@ -75,6 +75,24 @@ def test_row_stride(orc, layout):
     assert torch.all(out[:, 384:] == 7.0)
 
 
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_dequantize_to_16_byte_aligned_destinations(orc, layout):
+    """Destinations 16- but not 32-byte aligned (and a row stride of 8 mod 16
+    elements) take the two-store path; the bytes must not change."""
+    g = torch.Generator().manual_seed(13)
+    x = torch.randn(130, 272, generator=g).to(torch.bfloat16)
+    q = nv.quantize(x.cuda(), sf_layout=layout)
+    codes, sf, st = assert_quant_equal(orc, q, bits(x), layout)
+    ref = orc.dequantize(codes, sf, st)
+    buf = torch.empty(130 * 272 + 8, dtype=torch.bfloat16, device="cuda")
+    flat = buf[8:].view(130, 272)  # base 16 bytes past a 256-byte boundary
+    nv.dequantize(q, out=flat)
+    np.testing.assert_array_equal(bits(flat), ref)
+    wide = torch.empty(130 * 280 + 8, dtype=torch.bfloat16, device="cuda")[8:].view(130, 280)
+    nv.dequantize(q, out=wide[:, :272])  # ld = 280
+    np.testing.assert_array_equal(bits(wide[:, :272]), ref)
+
+
 def test_given_tensor_scale(orc):
     g = torch.Generator().manual_seed(4)
     x = (torch.randn(96, 160, generator=g) * 5).to(torch.bfloat16)

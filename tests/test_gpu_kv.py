@@ -91,6 +91,23 @@ def test_small_geometries(orc, tpf, heads, hd, nf):
     np.testing.assert_array_equal(bits(ko), ref)
 
 
+def test_window_into_16_byte_aligned_outputs(orc):
+    tpf, heads, hd = 9, 2, 32
+    g = torch.Generator().manual_seed(17)
+    k = (torch.randn(3 * tpf, heads, hd, generator=g)).to(torch.bfloat16)
+    cache = nv.KVCache(4, tpf, heads, hd)
+    cache.quant_chunk(k.cuda(), k.cuda(), [3, 1, 0])
+    n = 3 * tpf * heads * hd
+    kb = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")[8:].view(3 * tpf, heads, hd)
+    vb = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")[8:].view(3 * tpf, heads, hd)
+    window = [0, 3, 1]
+    cache.dequant_window(window, kb, vb)
+    ref = orc.kv_dequant_window(np_u8(cache.k_codes), np_u8(cache.k_sf), cache.k_st.cpu().numpy(),
+                                window, tpf, heads, hd)
+    np.testing.assert_array_equal(bits(kb), ref)
+    np.testing.assert_array_equal(bits(vb), ref)
+
+
 def test_bad_slots_rejected_on_host():
     cache = nv.KVCache(4, 8, 2, 16)
     k = torch.zeros(16, 2, 16, dtype=torch.bfloat16, device="cuda")
