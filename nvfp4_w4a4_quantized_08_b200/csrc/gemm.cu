@@ -12,15 +12,21 @@
 //   warp 0      TMA producer: 2-D tensor copies of the A and W code tiles
 //               (128-byte K slabs, 128-byte swizzle) and 1-D bulk copies of the
 //               matching 512-byte scale tiles into a 3-stage shared-memory ring.
-//   warp 1      tensor-core issuer: per K = 64 step, copies that step's scales
-//               into tensor memory (tcgen05.cp, interleaved with the MMAs) and
-//               issues one MMA; it also owns the tensor-memory allocation.
+//   warp 1      tensor-core issuer: one MMA per K = 64 step once that step's
+//               scales are in tensor memory; it also owns the tensor-memory
+//               allocation.
 //   warps 2..5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
 //               s_tA * s_tW, round to bf16 / fp32, stage in swizzled shared
 //               memory, TMA tensor store (rows past M are clipped by the store).
-// Two accumulators overlap in tensor memory (columns [0,256) and [192,448)):
-// the epilogue reads the 64 shared columns of a tile first and releases them,
-// so the next tile's MMAs run while it drains the other 192 columns.
+//   warps 6..9  scale writers: per K step, each writes the scale words its lane
+//               quadrant reads into a ring of 5 tensor-memory scale slots
+//               (tcgen05.st), off the tensor pipe, which would otherwise run
+//               the scale copies (tcgen05.cp) and the MMAs one after the other.
+// Tensor memory: the 128 x 256 FP32 accumulator in columns [0,256) and a ring
+// of 21 scale slots (12 columns each) in [256,508).  The epilogue reads the
+// whole accumulator into registers and releases it before its stores, so the
+// tensor pipe idles only for that read-out between tiles; the deep scale ring
+// lets the scale writers run far enough ahead that the MMAs never wait on them.
 // Every spin-wait is bounded (wait_limit_ns).  A wait that runs out records
 // NVFP4_ERR_TIMEOUT, raises a CTA-wide abort flag, and the CTA drains its own
 // copies, MMAs and stores in flight before freeing tensor memory and returning.
@@ -44,11 +50,12 @@ constexpr int kABytes = kBM * kBKBytes;      // 16 KB
 constexpr int kBBytes = kBN * kBKBytes;      // 32 KB
 constexpr int kSfaBytes = 4 * 512;           // 4 scale tiles of 128 rows x 4 blocks
 constexpr int kSfbBytes = 2 * 4 * 512;       // 2 row tiles of W
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;
-constexpr int kAcc1Col = 192;                // second accumulator; [192,256) shared
-constexpr int kOverlapCols = 256 - kAcc1Col;
-constexpr int kSfCol = 448;                  // per K step j: SFA at +12j, SFB at +12j+4
+constexpr int kSfCol = kBN;                  // scale sets after the accumulator
+constexpr int kSfSets = 4;                   // stages of scales resident in tensor memory
+constexpr int kSfStepCols = 12;              // per K step: SFA at +0, SFB at +4 and +8
+constexpr int kSfSetCols = kKSteps * kSfStepCols;
 constexpr int kStageBufBytes = 32 * 128;     // epilogue staging: 32 rows x 128 bytes
 constexpr int kEpiWarps = 4;
 
@@ -59,12 +66,15 @@ constexpr int kOffSfa = kOffB + kStages * kBBytes;
 constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
 constexpr int kOffStage = kOffSfb + kStages * kSfbBytes;            // 1024-aligned
 constexpr int kOffBar = kOffStage + kEpiWarps * 2 * kStageBufBytes;
-constexpr int kNumBars = 2 * kStages + 4;  // full[], empty[], acc_full[2], acc_release, drain
+// full[], empty[], acc_full, (unused), acc_release, drain, sf_free[]
+constexpr int kNumBars = 2 * kStages + 4 + kSfSets;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
 constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
 static_assert(kOffStage % 1024 == 0, "staging buffers need 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kSfCol + kSfSets * kSfSetCols <= kTmemCols, "tensor memory budget");
+static_assert(kBN <= kSfCol, "the accumulator overlaps the scale slots");
 
 // Instruction descriptor, block-scaled kinds: E2M1 A and B (format 1 at bits
 // 7-9 and 10-12), K-major both, N >> 3 at bits 17-22, E4M3 scales (bit 23 = 0),
@@ -149,17 +159,6 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-// Descriptor of a 32-row x 16-byte scale tile (no swizzle; 8-row core
-// matrices of 128 bytes, 128 bytes apart), the source of tcgen05.cp 32x128b.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
-  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t(128 >> 4) << 32) | (uint64_t(1) << 46);
-}
-
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                        uint32_t accumulate) {
@@ -184,6 +183,50 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Named barriers 1..kSfSets hand a stage's scales from the 4 writer warps
+// (arrive) to the issuer warp (sync).
+constexpr int kNamedBarThreads = 5 * 32;
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// One 32-bit column of this warp's 32 tensor-memory lanes from a register.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v)
+               : "memory");
+}
+
+// Four consecutive 32-bit columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // ---------------------------------------------------------------- bounded waits
@@ -244,6 +287,30 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// One 128-byte segment of each of this warp's 32 output rows (32 words a
+// lane) through the warp's staging buffer (two alternating 4 KB buffers,
+// 128-byte swizzle) and a TMA tensor store at column x, row y.
+__device__ __forceinline__ void store_row_chunk(const uint32_t (&w)[32], uint32_t stage0,
+                                                uint32_t& nstore, int lane, const CUtensorMap* map,
+                                                int32_t x, int32_t y) {
+  const uint32_t sb = stage0 + (nstore & 1) * kStageBufBytes;
+  // the store issued two chunks ago must have finished reading this buffer
+  if (lane == 0) bulk_wait_read_le1();
+  __syncwarp();
+  const uint32_t row = sb + uint32_t(lane) * 128;
+  const uint32_t sw = uint32_t(lane) & 7;  // 128-byte swizzle: 16-byte unit ^ (row % 8)
+#pragma unroll
+  for (uint32_t u = 0; u < 8; ++u)
+    st_shared_v4(row + ((u ^ sw) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, x, y, sb);
+    bulk_commit();
+  }
+  ++nstore;
+}
+
 struct Params {
   const uint8_t* a_sf;
   const uint8_t* w_sf;
@@ -272,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_acc_full = bar_empty + 8 * kStages;     // + 8 b
   const uint32_t bar_acc_release = bar_acc_full + 16;
   const uint32_t bar_drain = bar_acc_release + 8;
+  const uint32_t bar_sf_free = bar_drain + 8;                // + 8 set
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
@@ -284,9 +352,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bar_init(bar_empty + 8 * s, 1);
     }
     bar_init(bar_acc_full, 1);
-    bar_init(bar_acc_full + 8, 1);
     bar_init(bar_acc_release, kEpiWarps);
     bar_init(bar_drain, 1);
+    for (int s = 0; s < kSfSets; ++s) bar_init(bar_sf_free + 8 * s, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -342,51 +410,97 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0, local = 0;
-      bool ok = true;
-      for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
-        // the previous tile's epilogue must have read the columns the two
-        // accumulators share (and, before that, all of the tile before it)
-        if (local > 0 && !waiter.wait(bar_acc_release, (local - 1) & 1)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + ((local & 1) ? kAcc1Col : 0);
-        for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
-          if (!waiter.wait(bar_full + 8 * stage, phase)) { ok = false; break; }
+    // The whole warp takes part in the waits and the named-barrier handoff
+    // from the scale writers; lane 0 issues.  Every writer arrives once per
+    // stage, aborting or not, so the bar.sync below always completes.
+    uint32_t stage = 0, phase = 0, set = 0, local = 0;
+    bool ok = true;
+    for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+      // the previous tile's epilogue must have read the accumulator out
+      if (local > 0 && !__all_sync(0xFFFFFFFFu, waiter.wait(bar_acc_release, (local - 1) & 1)))
+        break;
+      for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
+        if (!__all_sync(0xFFFFFFFFu, waiter.wait(bar_full + 8 * stage, phase))) { ok = false; break; }
+        // this stage's scales are in tensor memory set `set`
+        named_bar_sync(1 + set, kNamedBarThreads);
+        if (*abort_flag) { ok = false; break; }
+        if (lane == 0) {
           tc_fence_after();
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
-          const uint32_t sfa_s = sbase + kOffSfa + stage * kSfaBytes;
-          const uint32_t sfb_s = sbase + kOffSfb + stage * kSfbBytes;
           const uint32_t a_s = sbase + kOffA + stage * kABytes;
           const uint32_t b_s = sbase + kOffB + stage * kBBytes;
-          for (uint32_t j = 0; j < nk; ++j) {
-            // scales of this K step, then its MMA (tcgen05 ops issue in order)
-            const uint32_t sf_col = tmem + kSfCol + 12 * j;
-            tc_cp_sf(sf_col, desc_sf(sfa_s + 512 * j));
-            tc_cp_sf(sf_col + 4, desc_sf(sfb_s + 512 * j));
-            tc_cp_sf(sf_col + 8, desc_sf(sfb_s + 2048 + 512 * j));
-            tc_mma(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), kIdesc, sf_col,
-                   sf_col + 4, (kb | j) != 0);
-          }
+          const uint32_t sf = tmem + kSfCol + kSfSetCols * set;
+          for (uint32_t j = 0; j < nk; ++j)
+            tc_mma(tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), kIdesc,
+                   sf + kSfStepCols * j, sf + kSfStepCols * j + 4, (kb | j) != 0);
+          tc_commit(bar_sf_free + 8 * set);  // the set is free once these MMAs complete
           tc_commit(bar_empty + 8 * stage);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
-        if (!ok) break;
-        tc_commit(bar_acc_full + 8 * (local & 1));
+        __syncwarp();
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (++set == kSfSets) set = 0;
       }
-      // drain: every tcgen05 operation this thread issued has completed
+      if (!ok) break;
+      if (lane == 0) tc_commit(bar_acc_full);
+      __syncwarp();
+    }
+    // drain: every tcgen05 operation this warp issued has completed
+    if (lane == 0) {
       tc_commit(bar_drain);
       drain_wait(bar_drain, 0, p.status);
     }
+    __syncwarp();
+  } else if (warp >= 2 + kEpiWarps) {
+    // ------------------------------------------------------------ scale writers
+    // Each warp owns one tensor-memory lane quadrant q; lane quadrant q of the
+    // tensor core computes output rows 32q..32q+31.  A staged scale tile is 32
+    // chunks of 16 bytes, chunk l holding the four E4M3 scales of rows l,
+    // l+32, l+64, l+96 of a 128-row operand tile.  Per K step the MMA reads
+    //   A scales of row 32q + l: lane 32q + l, column sfa + q (its own rows);
+    //   W scales of row n (any of the 256, every quadrant needs them all):
+    //     lane 32q + n % 32, column sfb + n / 32.
+    // So warp q writes word q of A chunk `lane` into one column and both W
+    // chunks `lane` whole (4 columns each) into its lanes, a stage at a time,
+    // then hands the set to the issuer through named barrier 1 + set.  The
+    // writers run up to kSfSets stages ahead of the MMAs.
+    const uint32_t q = uint32_t(warp & 3);
+    const uint32_t lane_bits = (q * 32) << 16;
+    uint32_t stage = 0, phase = 0, set = 0, set_phase = 0;
+    bool ok = true;
+    for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
+        ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_full + 8 * stage, phase)) &&
+             __all_sync(0xFFFFFFFFu, waiter.wait(bar_sf_free + 8 * set, set_phase ^ 1));
+        if (ok) {
+          tc_fence_after();
+          const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
+          const uint32_t sfa_s = sbase + kOffSfa + stage * kSfaBytes + 16 * uint32_t(lane) + 4 * q;
+          const uint32_t sfb_s = sbase + kOffSfb + stage * kSfbBytes + 16 * uint32_t(lane);
+          const uint32_t col = tmem + lane_bits + kSfCol + kSfSetCols * set;
+          for (uint32_t j = 0; j < nk; ++j) {
+            tmem_st1(col + kSfStepCols * j + q, ld_shared_u32(sfa_s + 512 * j));
+            tmem_st4(col + kSfStepCols * j + 4, ld_shared_v4(sfb_s + 512 * j));
+            tmem_st4(col + kSfStepCols * j + 8, ld_shared_v4(sfb_s + 2048 + 512 * j));
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          tc_fence_before();
+        }
+        // arrive even when aborting: the issuer is (or will be) waiting here
+        named_bar_arrive(1 + set, kNamedBarThreads);
+        if (!ok) break;
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (++set == kSfSets) { set = 0; set_phase ^= 1; }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
+    // The accumulator is read out whole into registers (bf16: 128 packed words
+    // a thread; fp32: two halves of 128 words) and released to the MMA issuer
+    // before the stores, so the next tile's MMAs wait only for the reads.
     const uint32_t ew = uint32_t(warp - 2);            // staging buffers of this warp
     const uint32_t quad = uint32_t(warp & 3);          // tensor-memory lane quadrant
     const float alpha = __fmul_rn(*p.a_st, *p.w_st);
     const bool bf16 = p.c_dtype == NVFP4_BF16;
-    const uint32_t chunk_cols = bf16 ? 64 : 32;        // 128-byte rows in staging
-    const uint32_t nchunks = kBN / chunk_cols;
-    const uint32_t overlap_chunks = kOverlapCols / chunk_cols;
     const uint32_t stage0 = sbase + kOffStage + ew * 2 * kStageBufBytes;
     uint32_t local = 0, nstore = 0;
     // running max of |stored value| as magnitude bits: two bf16 halves, or fp32
@@ -396,69 +510,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tm = t % p.tiles_m, tn = t / p.tiles_m;
       // accumulator lanes past the last row of C hold zeros; leave them out anyway
       const bool row_live = want_max && tm * kBM + quad * 32 + uint32_t(lane) < p.M;
-      const uint32_t buf = local & 1;
+      const int32_t y = int32_t(tm * kBM + quad * 32);
       // warp-uniform outcome: tcgen05.ld below is .sync.aligned
-      const bool ok = waiter.wait(bar_acc_full + 8 * buf, (local >> 1) & 1);
+      const bool ok = waiter.wait(bar_acc_full, local & 1);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + ((quad * 32) << 16) + (buf ? kAcc1Col : 0);
-      // the shared columns first: the last 64 of accumulator 0, the first 64 of 1
-      const uint32_t first = buf ? 0 : nchunks - overlap_chunks;
+      const uint32_t taddr = tmem + ((quad * 32) << 16);
+      if (bf16) {
+        uint32_t pk[128];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[32];
+          tmem_ld32(taddr + 32 * c, r);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[16 * c + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
+                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(bar_acc_release);
+        if (row_live) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) vmax = __vmaxu2(vmax, pk[e] & 0x7FFF7FFFu);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          store_row_chunk(*reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * ch]), stage0, nstore,
+                          lane, &map_c, int32_t(tn * kBN + 64 * ch), y);
+      } else {
 #pragma unroll 1
-      for (uint32_t i = 0; i < nchunks; ++i) {
-        const uint32_t c = (first + i) % nchunks;
-        uint32_t r[64];
-        tmem_ld32(taddr + c * chunk_cols, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        if (bf16)
-          tmem_ld32(taddr + c * chunk_cols + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        if (i + 1 == overlap_chunks) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) bar_arrive(bar_acc_release);
-        }
-        // staging buffer: wait until the store issued two chunks ago has read it
-        const uint32_t sb = stage0 + (nstore & 1) * kStageBufBytes;
-        if (lane == 0) bulk_wait_read_le1();
-        __syncwarp();
-        const uint32_t row = sb + uint32_t(lane) * 128;
-        const uint32_t sw = uint32_t(lane) & 7;  // 128-byte swizzle: 16-byte unit ^ (row % 8)
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[128];
 #pragma unroll
-        for (uint32_t u = 0; u < 8; ++u) {
-          uint32_t w0, w1, w2, w3;
-          if (bf16) {
-            float f[8];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(taddr + 128 * half + 32 * c, r);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(__uint_as_float(r[8 * u + e]), alpha);
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(f[0], f[1]);
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(f[2], f[3]);
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(f[4], f[5]);
-            __nv_bfloat162 b3 = __floats2bfloat162_rn(f[6], f[7]);
-            w0 = *reinterpret_cast<uint32_t*>(&b0);
-            w1 = *reinterpret_cast<uint32_t*>(&b1);
-            w2 = *reinterpret_cast<uint32_t*>(&b2);
-            w3 = *reinterpret_cast<uint32_t*>(&b3);
-            if (row_live)
-              vmax = __vmaxu2(__vmaxu2(vmax, __vmaxu2(w0 & 0x7FFF7FFFu, w1 & 0x7FFF7FFFu)),
-                              __vmaxu2(w2 & 0x7FFF7FFFu, w3 & 0x7FFF7FFFu));
-          } else {
-            w0 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 0]), alpha));
-            w1 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 1]), alpha));
-            w2 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 2]), alpha));
-            w3 = __float_as_uint(__fmul_rn(__uint_as_float(r[4 * u + 3]), alpha));
-            if (row_live)
-              vmax = max(max(vmax, max(w0 & 0x7FFFFFFFu, w1 & 0x7FFFFFFFu)),
-                         max(w2 & 0x7FFFFFFFu, w3 & 0x7FFFFFFFu));
+            for (int e = 0; e < 32; ++e)
+              v[32 * c + e] = __float_as_uint(__fmul_rn(__uint_as_float(r[e]), alpha));
           }
-          st_shared_v4(row + ((u ^ sw) << 4), w0, w1, w2, w3);
+          if (half == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) bar_arrive(bar_acc_release);
+          }
+          if (row_live) {
+#pragma unroll
+            for (int e = 0; e < 128; ++e) vmax = max(vmax, v[e] & 0x7FFFFFFFu);
+          }
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+            store_row_chunk(*reinterpret_cast<const uint32_t(*)[32]>(&v[32 * ch]), stage0,
+                            nstore, lane, &map_c, int32_t(tn * kBN + 128 * half + 32 * ch), y);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&map_c, int32_t(tn * kBN + c * chunk_cols), int32_t(tm * kBM + quad * 32),
-                       sb);
-          bulk_commit();
-        }
-        ++nstore;
       }
     }
     if (want_max) {
