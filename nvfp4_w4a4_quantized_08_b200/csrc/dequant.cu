@@ -110,6 +110,8 @@ __device__ __forceinline__ void store_block(uint8_t* dst, uint4 lo, uint4 hi) {
 // load the last block again and store nothing.
 template <int kSfLayout, bool kContig, bool kWide>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(DequantArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const float s_t = *a.s_t;
   const uint32_t stride = gridDim.x * blockDim.x;
   for (uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x; b0 < a.blocks;
@@ -151,6 +153,8 @@ struct KvDequantArgs {
 
 template <bool kWide>
 __global__ void __launch_bounds__(kDqThreads) kv_dequant_kernel(KvDequantArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int plane = blockIdx.y;
   const uint8_t* codes = plane == 0 ? a.codes[0] : a.codes[1];
   const uint8_t* sfp = plane == 0 ? a.sf[0] : a.sf[1];
@@ -213,26 +217,21 @@ cudaError_t launch_dequantize(const LaunchDequant& d, cudaStream_t st) {
   const bool mma = d.sf_layout == NVFP4_SF_MMA128x4;
   const bool wide = reinterpret_cast<uintptr_t>(d.out) % 32 == 0 && (contig || d.ld % 16 == 0);
   auto launch = [&](auto kernel) {
-    kernel<<<dq_grid(kernel, a.blocks, d.sm_count, 1), kDqThreads, 0, st>>>(a);
+    return launch_pdl(kernel, dim3(dq_grid(kernel, a.blocks, d.sm_count, 1)), dim3(kDqThreads), 0,
+                      st, a);
   };
   if (wide) {
-    if (mma) {
-      if (contig) launch(dequant_kernel<NVFP4_SF_MMA128x4, true, true>);
-      else launch(dequant_kernel<NVFP4_SF_MMA128x4, false, true>);
-    } else {
-      if (contig) launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true, true>);
-      else launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false, true>);
-    }
-  } else {
-    if (mma) {
-      if (contig) launch(dequant_kernel<NVFP4_SF_MMA128x4, true, false>);
-      else launch(dequant_kernel<NVFP4_SF_MMA128x4, false, false>);
-    } else {
-      if (contig) launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true, false>);
-      else launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false, false>);
-    }
+    if (mma)
+      return contig ? launch(dequant_kernel<NVFP4_SF_MMA128x4, true, true>)
+                    : launch(dequant_kernel<NVFP4_SF_MMA128x4, false, true>);
+    return contig ? launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true, true>)
+                  : launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false, true>);
   }
-  return cudaGetLastError();
+  if (mma)
+    return contig ? launch(dequant_kernel<NVFP4_SF_MMA128x4, true, false>)
+                  : launch(dequant_kernel<NVFP4_SF_MMA128x4, false, false>);
+  return contig ? launch(dequant_kernel<NVFP4_SF_ROWMAJOR, true, false>)
+                : launch(dequant_kernel<NVFP4_SF_ROWMAJOR, false, false>);
 }
 
 cudaError_t launch_kv_dequant(const LaunchKvDequant& d, cudaStream_t st) {
@@ -250,12 +249,10 @@ cudaError_t launch_kv_dequant(const LaunchKvDequant& d, cudaStream_t st) {
                     reinterpret_cast<uintptr_t>(d.v_out) % 32 == 0;
   if (wide) {
     const int grid = dq_grid(kv_dequant_kernel<true>, a.blocks, d.sm_count, 2);
-    kv_dequant_kernel<true><<<dim3(grid, 2), kDqThreads, 0, st>>>(a);
-  } else {
-    const int grid = dq_grid(kv_dequant_kernel<false>, a.blocks, d.sm_count, 2);
-    kv_dequant_kernel<false><<<dim3(grid, 2), kDqThreads, 0, st>>>(a);
+    return launch_pdl(kv_dequant_kernel<true>, dim3(grid, 2), dim3(kDqThreads), 0, st, a);
   }
-  return cudaGetLastError();
+  const int grid = dq_grid(kv_dequant_kernel<false>, a.blocks, d.sm_count, 2);
+  return launch_pdl(kv_dequant_kernel<false>, dim3(grid, 2), dim3(kDqThreads), 0, st, a);
 }
 
 }  // namespace nvfp4

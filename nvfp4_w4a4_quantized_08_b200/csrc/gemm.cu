@@ -18,15 +18,15 @@
 //   warps 2..5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
 //               s_tA * s_tW, round to bf16 / fp32, stage in swizzled shared
 //               memory, TMA tensor store (rows past M are clipped by the store).
-//   warps 6..9  scale writers: per K step, each writes the scale words its lane
-//               quadrant reads into a ring of 5 tensor-memory scale slots
+//   warps 6..9  scale writers: per stage, each writes the scale words its lane
+//               quadrant reads into that stage's tensor-memory scale set
 //               (tcgen05.st), off the tensor pipe, which would otherwise run
-//               the scale copies (tcgen05.cp) and the MMAs one after the other.
-// Tensor memory: the 128 x 256 FP32 accumulator in columns [0,256) and a ring
-// of 21 scale slots (12 columns each) in [256,508).  The epilogue reads the
+//               the scale copies (tcgen05.cp) and the MMAs one after the other,
+//               and hands the set to the issuer through a named barrier.
+// Tensor memory: the 128 x 256 FP32 accumulator in columns [0,256) and one
+// 48-column scale set per shared-memory stage after it.  The epilogue reads the
 // whole accumulator into registers and releases it before its stores, so the
-// tensor pipe idles only for that read-out between tiles; the deep scale ring
-// lets the scale writers run far enough ahead that the MMAs never wait on them.
+// tensor pipe idles only for that read-out between tiles.
 // Every spin-wait is bounded (wait_limit_ns).  A wait that runs out records
 // NVFP4_ERR_TIMEOUT, raises a CTA-wide abort flag, and the CTA drains its own
 // copies, MMAs and stores in flight before freeing tensor memory and returning.
@@ -53,7 +53,7 @@ constexpr int kSfbBytes = 2 * 4 * 512;       // 2 row tiles of W
 constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;
 constexpr int kSfCol = kBN;                  // scale sets after the accumulator
-constexpr int kSfSets = 4;                   // stages of scales resident in tensor memory
+constexpr int kSfSets = kStages;             // one scale set per shared-memory stage
 constexpr int kSfStepCols = 12;              // per K step: SFA at +0, SFB at +4 and +8
 constexpr int kSfSetCols = kKSteps * kSfStepCols;
 constexpr int kStageBufBytes = 32 * 128;     // epilogue staging: 32 rows x 128 bytes
@@ -66,8 +66,8 @@ constexpr int kOffSfa = kOffB + kStages * kBBytes;
 constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
 constexpr int kOffStage = kOffSfb + kStages * kSfbBytes;            // 1024-aligned
 constexpr int kOffBar = kOffStage + kEpiWarps * 2 * kStageBufBytes;
-// full[], empty[], acc_full, (unused), acc_release, drain, sf_free[]
-constexpr int kNumBars = 2 * kStages + 4 + kSfSets;
+// full[], empty[], acc_full, (unused), acc_release, drain
+constexpr int kNumBars = 2 * kStages + 4;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
 constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
@@ -339,7 +339,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_acc_full = bar_empty + 8 * kStages;     // + 8 b
   const uint32_t bar_acc_release = bar_acc_full + 16;
   const uint32_t bar_drain = bar_acc_release + 8;
-  const uint32_t bar_sf_free = bar_drain + 8;                // + 8 set
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
@@ -354,7 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     bar_init(bar_acc_full, 1);
     bar_init(bar_acc_release, kEpiWarps);
     bar_init(bar_drain, 1);
-    for (int s = 0; s < kSfSets; ++s) bar_init(bar_sf_free + 8 * s, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -370,6 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
+  // on-chip setup done; from here on global memory is read and written
+  pdl_wait();
+  pdl_trigger();
 
   const Waiter waiter{p.wait_limit_ns, abort_flag, p.status};
   const uint32_t num_tiles = p.tiles_m * p.tiles_n;
@@ -410,35 +411,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // The whole warp takes part in the waits and the named-barrier handoff
-    // from the scale writers; lane 0 issues.  Every writer arrives once per
-    // stage, aborting or not, so the bar.sync below always completes.
-    uint32_t stage = 0, phase = 0, set = 0, local = 0;
+    // Lane 0 issues; the whole warp takes part in the named-barrier handoff
+    // from the scale writers (bar.sync counts whole warps).  The MMAs of a
+    // stage hold the issuing thread until the tensor pipe accepts them, so
+    // everything between two stages is kept short: one handoff, one commit.
+    // Every writer arrives once per stage, aborting or not, so the bar.sync
+    // below always completes.
+    uint32_t stage = 0, phase = 0, local = 0;
     bool ok = true;
     for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
       // the previous tile's epilogue must have read the accumulator out
-      if (local > 0 && !__all_sync(0xFFFFFFFFu, waiter.wait(bar_acc_release, (local - 1) & 1)))
-        break;
+      if (local > 0) {
+        bool released = true;
+        if (lane == 0) released = waiter.wait(bar_acc_release, (local - 1) & 1);
+        if (!__shfl_sync(0xFFFFFFFFu, released, 0)) break;
+      }
       for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
-        if (!__all_sync(0xFFFFFFFFu, waiter.wait(bar_full + 8 * stage, phase))) { ok = false; break; }
-        // this stage's scales are in tensor memory set `set`
-        named_bar_sync(1 + set, kNamedBarThreads);
+        // the writers have seen this stage land and put its scales in set `stage`
+        named_bar_sync(1 + stage, kNamedBarThreads);
         if (*abort_flag) { ok = false; break; }
-        if (lane == 0) {
+        // complete already (the writers waited for it); observed here too, as
+        // the MMAs read the stage's operands
+        if (lane == 0 && waiter.wait(bar_full + 8 * stage, phase)) {
           tc_fence_after();
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
-          const uint32_t a_s = sbase + kOffA + stage * kABytes;
-          const uint32_t b_s = sbase + kOffB + stage * kBBytes;
-          const uint32_t sf = tmem + kSfCol + kSfSetCols * set;
-          for (uint32_t j = 0; j < nk; ++j)
-            tc_mma(tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), kIdesc,
-                   sf + kSfStepCols * j, sf + kSfStepCols * j + 4, (kb | j) != 0);
-          tc_commit(bar_sf_free + 8 * set);  // the set is free once these MMAs complete
+          const uint64_t a_d = desc_sw128(sbase + kOffA + stage * kABytes);
+          const uint64_t b_d = desc_sw128(sbase + kOffB + stage * kBBytes);
+          const uint32_t sf = tmem + kSfCol + kSfSetCols * stage;
+          for (uint32_t j = 0; j < nk; ++j)  // K step j: +32 bytes = +2 in the address field
+            tc_mma(tmem, a_d + 2 * j, b_d + 2 * j, kIdesc, sf + kSfStepCols * j,
+                   sf + kSfStepCols * j + 4, (kb | j) != 0);
+          // frees the shared-memory stage and its scale set once these MMAs complete
           tc_commit(bar_empty + 8 * stage);
         }
         __syncwarp();
         if (++stage == kStages) { stage = 0; phase ^= 1; }
-        if (++set == kSfSets) set = 0;
       }
       if (!ok) break;
       if (lane == 0) tc_commit(bar_acc_full);
@@ -461,22 +468,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     //     lane 32q + n % 32, column sfb + n / 32.
     // So warp q writes word q of A chunk `lane` into one column and both W
     // chunks `lane` whole (4 columns each) into its lanes, a stage at a time,
-    // then hands the set to the issuer through named barrier 1 + set.  The
-    // writers run up to kSfSets stages ahead of the MMAs.
+    // into the stage's scale set, then hands it to the issuer through named
+    // barrier 1 + stage.  A set is free when its stage is full again: the
+    // producer refilled the stage after the MMAs that read the set completed.
     const uint32_t q = uint32_t(warp & 3);
     const uint32_t lane_bits = (q * 32) << 16;
-    uint32_t stage = 0, phase = 0, set = 0, set_phase = 0;
+    uint32_t stage = 0, phase = 0;
     bool ok = true;
     for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
-        ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_full + 8 * stage, phase)) &&
-             __all_sync(0xFFFFFFFFu, waiter.wait(bar_sf_free + 8 * set, set_phase ^ 1));
+        ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_full + 8 * stage, phase));
         if (ok) {
           tc_fence_after();
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
           const uint32_t sfa_s = sbase + kOffSfa + stage * kSfaBytes + 16 * uint32_t(lane) + 4 * q;
           const uint32_t sfb_s = sbase + kOffSfb + stage * kSfbBytes + 16 * uint32_t(lane);
-          const uint32_t col = tmem + lane_bits + kSfCol + kSfSetCols * set;
+          const uint32_t col = tmem + lane_bits + kSfCol + kSfSetCols * stage;
           for (uint32_t j = 0; j < nk; ++j) {
             tmem_st1(col + kSfStepCols * j + q, ld_shared_u32(sfa_s + 512 * j));
             tmem_st4(col + kSfStepCols * j + 4, ld_shared_v4(sfb_s + 512 * j));
@@ -486,10 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
         }
         // arrive even when aborting: the issuer is (or will be) waiting here
-        named_bar_arrive(1 + set, kNamedBarThreads);
+        named_bar_arrive(1 + stage, kNamedBarThreads);
         if (!ok) break;
         if (++stage == kStages) { stage = 0; phase ^= 1; }
-        if (++set == kSfSets) { set = 0; set_phase ^= 1; }
       }
     }
   } else {
@@ -672,9 +678,8 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.c_dtype = g.c_dtype;
   const uint32_t tiles = p.tiles_m * p.tiles_n;
   const int grid = int(tiles < uint32_t(g.sm_count) ? tiles : uint32_t(g.sm_count));
-  gemm::nvfp4_gemm_kernel<<<grid, gemm::kThreads, gemm::kSmemBytes, st>>>(map_a, map_w, map_c,
-                                                                          p);
-  return cudaGetLastError();
+  return launch_pdl(gemm::nvfp4_gemm_kernel, dim3(grid), dim3(gemm::kThreads),
+                    size_t(gemm::kSmemBytes), st, map_a, map_w, map_c, p);
 }
 
 }  // namespace nvfp4

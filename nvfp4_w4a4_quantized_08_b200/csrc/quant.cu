@@ -144,6 +144,8 @@ struct AmaxArgs {
 
 template <typename InT, bool kContig>
 __global__ void __launch_bounds__(kQuantThreads) amax_kernel(AmaxArgs args) {
+  pdl_wait();
+  pdl_trigger();
   const int plane = blockIdx.y;
   const InMap m = plane == 0 ? args.in[0] : args.in[1];
   const uint32_t blocks = m.units >> 1;
@@ -365,6 +367,9 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args)
   constexpr int D = Prefetch<InT>::kDepth;
   __shared__ float inv_tab[128];
   __shared__ float s_t_shared;
+  fill_inv_table(inv_tab);
+  pdl_wait();
+  pdl_trigger();
   const uint32_t stride = gridDim.x * blockDim.x;
   const uint32_t blocks = args.in.units >> 1;
   uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x;
@@ -375,7 +380,6 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args)
     load_block<InT>(block_ptr<InT, kContig>(args.in, min(b, blocks - 1)), cur[i]);
   }
   if (threadIdx.x == 0) s_t_shared = take_scale(args.s_t_in, args.amax_in, args.ws, 0);
-  fill_inv_table(inv_tab);
   __syncthreads();
   const float s_t = s_t_shared;
   const bool in_domain = tensor_scale_in_domain(s_t);
@@ -450,6 +454,9 @@ __global__ void __launch_bounds__(kQuantThreads, 4) kv_quant_kernel(KvQuantArgs 
   constexpr int D = Prefetch<__nv_bfloat16>::kDepth;
   __shared__ float inv_tab[128];
   __shared__ float s_t_shared;
+  fill_inv_table(inv_tab);
+  pdl_wait();
+  pdl_trigger();
   const int plane = blockIdx.y;
   const InMap m = plane == 0 ? args.in[0] : args.in[1];
   const uint32_t stride = gridDim.x * blockDim.x;
@@ -463,7 +470,6 @@ __global__ void __launch_bounds__(kQuantThreads, 4) kv_quant_kernel(KvQuantArgs 
                               cur[i]);
   }
   if (threadIdx.x == 0) s_t_shared = take_scale(nullptr, nullptr, args.ws, plane);
-  fill_inv_table(inv_tab);
   __syncthreads();
   const float s_t = s_t_shared;
   const bool in_domain = tensor_scale_in_domain(s_t);
@@ -526,24 +532,25 @@ static int wave_grid(uint32_t units, uint32_t per_thread, int per_sm, int sm_cou
 }
 
 template <typename InT, bool kContig>
-static void launch_amax(const AmaxArgs& aa, int planes, int sm_count, cudaStream_t st) {
+static cudaError_t launch_amax(const AmaxArgs& aa, int planes, int sm_count, cudaStream_t st) {
   static const int per_sm = resident_per_sm(amax_kernel<InT, kContig>);
   const int grid = wave_grid(aa.in[0].units, 2, per_sm, sm_count, planes);
-  amax_kernel<InT, kContig><<<dim3(grid, planes), kQuantThreads, 0, st>>>(aa);
+  return launch_pdl(amax_kernel<InT, kContig>, dim3(grid, planes), dim3(kQuantThreads), 0, st, aa);
 }
 
 template <typename InT, bool kContig, int kSfLayout>
-static void launch_encode(const QuantArgs& a, int sm_count, cudaStream_t st) {
+static cudaError_t launch_encode(const QuantArgs& a, int sm_count, cudaStream_t st) {
   static const int per_sm = resident_per_sm(quant_kernel<InT, kContig, kSfLayout>);
   const int grid = wave_grid(a.in.units, 1, per_sm, sm_count, 1);
-  quant_kernel<InT, kContig, kSfLayout><<<grid, kQuantThreads, 0, st>>>(a);
+  return launch_pdl(quant_kernel<InT, kContig, kSfLayout>, dim3(grid), dim3(kQuantThreads), 0, st,
+                    a);
 }
 
 template <bool kContig>
-static void launch_kv_encode(const KvQuantArgs& a, int sm_count, cudaStream_t st) {
+static cudaError_t launch_kv_encode(const KvQuantArgs& a, int sm_count, cudaStream_t st) {
   static const int per_sm = resident_per_sm(kv_quant_kernel<kContig>);
   const int grid = wave_grid(a.in[0].units, 1, per_sm, sm_count, 2);
-  kv_quant_kernel<kContig><<<dim3(grid, 2), kQuantThreads, 0, st>>>(a);
+  return launch_pdl(kv_quant_kernel<kContig>, dim3(grid, 2), dim3(kQuantThreads), 0, st, a);
 }
 
 static InMap make_inmap(const void* x, int64_t rows_total, int64_t cols, int64_t rows_per_group,
@@ -567,10 +574,9 @@ static cudaError_t launch_quant_t(const LaunchQuant& q, cudaStream_t st) {
     aa.in[0] = m;
     aa.in[1] = m;
     aa.ws = static_cast<uint32_t*>(q.ws);
-    if (contig)
-      launch_amax<InT, true>(aa, 1, q.sm_count, st);
-    else
-      launch_amax<InT, false>(aa, 1, q.sm_count, st);
+    const cudaError_t e = contig ? launch_amax<InT, true>(aa, 1, q.sm_count, st)
+                                 : launch_amax<InT, false>(aa, 1, q.sm_count, st);
+    if (e != cudaSuccess) return e;
   }
   QuantArgs a;
   a.in = m;
@@ -586,14 +592,11 @@ static cudaError_t launch_quant_t(const LaunchQuant& q, cudaStream_t st) {
   a.rows = uint32_t(q.rows);
   a.rows_pad = uint32_t((q.rows + 127) / 128 * 128);
   const bool mma = q.sf_layout == NVFP4_SF_MMA128x4;
-  if (contig) {
-    if (mma) launch_encode<InT, true, NVFP4_SF_MMA128x4>(a, q.sm_count, st);
-    else launch_encode<InT, true, NVFP4_SF_ROWMAJOR>(a, q.sm_count, st);
-  } else {
-    if (mma) launch_encode<InT, false, NVFP4_SF_MMA128x4>(a, q.sm_count, st);
-    else launch_encode<InT, false, NVFP4_SF_ROWMAJOR>(a, q.sm_count, st);
-  }
-  return cudaGetLastError();
+  if (contig)
+    return mma ? launch_encode<InT, true, NVFP4_SF_MMA128x4>(a, q.sm_count, st)
+               : launch_encode<InT, true, NVFP4_SF_ROWMAJOR>(a, q.sm_count, st);
+  return mma ? launch_encode<InT, false, NVFP4_SF_MMA128x4>(a, q.sm_count, st)
+             : launch_encode<InT, false, NVFP4_SF_ROWMAJOR>(a, q.sm_count, st);
 }
 
 cudaError_t launch_quantize(const LaunchQuant& q, cudaStream_t st) {
@@ -622,14 +625,11 @@ cudaError_t launch_kv_quant(const LaunchKvQuant& q, cudaStream_t st) {
   ka.bpf_div = make_fastdiv(ka.units_per_frame / 2);
   for (int f = 0; f < NVFP4_KV_MAX_CHUNK_FRAMES; ++f) ka.slots[f] = f < q.n_frames ? q.slots[f] : 0;
   ka.n_frames = q.n_frames;
-  if (contig) {
-    launch_amax<__nv_bfloat16, true>(aa, 2, q.sm_count, st);
-    launch_kv_encode<true>(ka, q.sm_count, st);
-  } else {
-    launch_amax<__nv_bfloat16, false>(aa, 2, q.sm_count, st);
-    launch_kv_encode<false>(ka, q.sm_count, st);
-  }
-  return cudaGetLastError();
+  cudaError_t e = contig ? launch_amax<__nv_bfloat16, true>(aa, 2, q.sm_count, st)
+                         : launch_amax<__nv_bfloat16, false>(aa, 2, q.sm_count, st);
+  if (e != cudaSuccess) return e;
+  return contig ? launch_kv_encode<true>(ka, q.sm_count, st)
+                : launch_kv_encode<false>(ka, q.sm_count, st);
 }
 
 }  // namespace nvfp4
