@@ -427,12 +427,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__shfl_sync(0xFFFFFFFFu, released, 0)) break;
       }
       for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
-        // the writers have seen this stage land and put its scales in set `stage`
+        // the writers have seen this stage land (they waited on its full
+        // barrier) and put its scales in set `stage`; the named barrier orders
+        // this thread after their observation
         named_bar_sync(1 + stage, kNamedBarThreads);
         if (*abort_flag) { ok = false; break; }
-        // complete already (the writers waited for it); observed here too, as
-        // the MMAs read the stage's operands
-        if (lane == 0 && waiter.wait(bar_full + 8 * stage, phase)) {
+        if (lane == 0) {
           tc_fence_after();
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
           const uint64_t a_d = desc_sw128(sbase + kOffA + stage * kABytes);

@@ -57,6 +57,29 @@ def test_small_shapes(orc, M, N, K):
     assert_gemm_close(y.cpu().numpy(), y_ref, S, False)
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_output_row_stride_and_alignment(orc, out_dtype):
+    """C written into a wider buffer (ldc = N + 8: rows 16- but not 32-byte
+    aligned, the 128-bit store path) and into one whose base is 16 bytes past
+    a 32-byte boundary; the columns outside [0, N) stay untouched."""
+    M, N, K = 200, 512, 256
+    g = torch.Generator().manual_seed(9)
+    a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    qa, qw, oa, ow = _operands(orc, a, w)
+    y_ref, S = orc.gemm(oa, ow)
+    wide = torch.full((M, N + 8), 3.0, dtype=out_dtype, device="cuda")
+    nv.gemm(qa, qw, out=wide[:, :N])
+    assert_gemm_close(wide[:, :N].float().cpu().numpy(), y_ref, S, out_dtype == torch.bfloat16)
+    assert torch.all(wide[:, N:] == 3.0)
+    shift = 16 // torch.tensor([], dtype=out_dtype).element_size()
+    buf = torch.zeros(M * N + shift, dtype=out_dtype, device="cuda")
+    y = buf[shift:].view(M, N)
+    nv.gemm(qa, qw, out=y)
+    assert_gemm_close(y.float().cpu().numpy(), y_ref, S, out_dtype == torch.bfloat16)
+    assert nv.device_status() == 0
+
+
 def test_qkv_projection(orc):
     """QKV projection: M=2640 (3 frames x 880 tokens), N=9216, K=3072; 32
     random rows plus the whole 80-row tail tile, all columns."""
