@@ -116,8 +116,9 @@ class Step:
         self.qf = nv.empty(M, F, device=device)
         self.ws = nv.workspace(device)
         # max|C| words handed from a GEMM epilogue to the quantization of its
-        # output: [0] down -> next layer's input, [1] out-proj, [2] FFN up
-        self.amax = torch.zeros(3, dtype=torch.float32, device=device)
+        # output: [0] down -> next layer's input, [1] out-proj, [2] FFN up,
+        # [3..5] the Q, K, V thirds of the QKV projection (K, V -> KV chunk)
+        self.amax = torch.zeros(6, dtype=torch.float32, device=device)
         self.new_slots = list(range(WINDOW, POOL))
         self.window = list(range(wl.SINK_FRAMES)) + \
             list(range(wl.SINK_FRAMES + NEW_FRAMES, WINDOW)) + self.new_slots
@@ -138,10 +139,12 @@ class Step:
             # layer 0's input has no producer in the step: it takes the amax pass
             nv.quantize(x, out=self.qa, ws=self.ws, amax_in=a_x if l > 0 else None)
             mk("gemm_qkv")
-            nv.gemm(self.qa, wq, out=self.qkv_out, ws=self.ws)
+            nv.gemm(self.qa, wq, out=self.qkv_out, ws=self.ws, c_amax=self.amax[3:6],
+                    c_amax_cols=D)
             mk("kv_quant")
             self.cache[l].quant_chunk(self.qkv_out[:, D:2 * D], self.qkv_out[:, 2 * D:],
-                                      self.new_slots, ws=self.ws)
+                                      self.new_slots, ws=self.ws, k_amax_in=self.amax[4:5],
+                                      v_amax_in=self.amax[5:6])
             mk("kv_dequant")
             self.cache[l].dequant_window(self.window, self.k_win, self.v_win)
             mk("quant_act")
@@ -163,9 +166,9 @@ class Step:
 
     # kernels launched per step: a quantize with its own amax pass 2 (layer 0's
     # input, the attention output), one fed by a GEMM's c_amax 1, gemm 1,
-    # kv_quant = amax + encode (2), kv_dequant 1
+    # kv_quant 1 (its amax comes from the QKV GEMM), kv_dequant 1
     def launches_per_step(self) -> int:
-        return self.layers * (2 + 1 + 1 + 1 + 4 * 1 + 2 + 1) + 1
+        return self.layers * (2 + 1 + 1 + 1 + 4 * 1 + 1 + 1) + 1
 
 
 # ---------------------------------------------------------------- clocks

@@ -173,18 +173,23 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64
  *      are masked).
  *   C: device, c_dtype (bf16 or fp32), row stride ldc >= N elements, ldc a
  *      multiple of 8, 16-byte aligned.
- *   c_amax: NULL, or a device float (4-byte aligned) into which the GEMM
+ *   c_amax: NULL, or device floats (4-byte aligned) into which the GEMM
  *      max-accumulates max|C| over the values as stored (after rounding to
  *      c_dtype), so that nvfp4_quantize(..., amax_in = c_amax, ...) can
- *      requantize C without an amax pass.  It must hold 0 (or a smaller
- *      non-negative value) before the call: zero-fill it once; the consuming
- *      quantize resets it.
+ *      requantize C without an amax pass.  With c_amax_cols == 0 there is one
+ *      word for all of C; with c_amax_cols > 0 (a multiple of 256 dividing N)
+ *      word g covers columns [g * c_amax_cols, (g + 1) * c_amax_cols), N /
+ *      c_amax_cols words in all: one per part of a fused output (for example
+ *      the Q, K and V thirds of a QKV projection, whose K and V words feed
+ *      nvfp4_kv_quant_chunk).  Every word must hold 0 (or a smaller
+ *      non-negative value) before the call: zero-fill them once; a consuming
+ *      quantize resets the words it reads.
  *   ws: device workspace (status word for the bounded waits).
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, ARCH, CUDA;
  * TIMEOUT via the status word. */
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C,
-                                  int32_t c_dtype, int64_t ldc, float* c_amax, void* ws,
-                                  size_t ws_bytes, void* stream);
+                                  int32_t c_dtype, int64_t ldc, float* c_amax,
+                                  int64_t c_amax_cols, void* ws, size_t ws_bytes, void* stream);
 
 /* Quantize one chunk of n_frames (1..8) new latent frames of K and V into the
  * cache.  The chunk is one NVFP4 tensor per K and per V: one s_t over the whole
@@ -195,12 +200,19 @@ NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, 
  *         token (token_stride >= heads * head_dim, a multiple of 8); this reads
  *         K and V straight out of a fused QKV projection output.
  *   dst_slots: host, n_frames distinct slot ids in [0, n_slots).
+ *   k_amax_in, v_amax_in: both NULL (the call runs an amax pass over K and V),
+ *         or both device floats (4-byte aligned) holding max|K| and max|V| of
+ *         the chunk as accumulated by the producer (nvfp4_gemm's per-column-
+ *         group c_amax over the K and V parts of a QKV output); the amax pass
+ *         is skipped and both words are reset to 0 when the call is done.
  *   ws: device workspace.
- * Errors: INVALID_ARG (slot ids out of range or repeated), UNSUPPORTED_SHAPE,
- * MISALIGNED, WORKSPACE, ARCH, CUDA; DOMAIN via the status word. */
+ * Errors: INVALID_ARG (slot ids out of range or repeated, one amax pointer
+ * without the other), UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, ARCH, CUDA;
+ * DOMAIN via the status word. */
 NVFP4_API nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const void* k, const void* v,
                                   int64_t token_stride, const int32_t* dst_slots, int32_t n_frames,
-                                  void* ws, size_t ws_bytes, void* stream);
+                                  float* k_amax_in, float* v_amax_in, void* ws, size_t ws_bytes,
+                                  void* stream);
 
 /* Rebuild contiguous bf16 K and V for attention from a list of slots, in list
  * order (for example 3 sink frames followed by the 9 window frames).

@@ -84,10 +84,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_dequantize.restype = i32
         L.nvfp4_dequantize.argtypes = [TP, vp, i64, vp]
         L.nvfp4_gemm.restype = i32
-        L.nvfp4_gemm.argtypes = [TP, TP, vp, i32, i64, vp, vp, sz, vp]
+        L.nvfp4_gemm.argtypes = [TP, TP, vp, i32, i64, vp, i64, vp, sz, vp]
         L.nvfp4_kv_quant_chunk.restype = i32
         L.nvfp4_kv_quant_chunk.argtypes = [KP, vp, vp, i64, ctypes.POINTER(ctypes.c_int32), i32,
-                                           vp, sz, vp]
+                                             vp, vp, vp, sz, vp]
         L.nvfp4_kv_dequant_window.restype = i32
         L.nvfp4_kv_dequant_window.argtypes = [KP, ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
         L.nvfp4_get_device_status.restype = i32

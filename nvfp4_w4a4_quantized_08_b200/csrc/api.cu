@@ -155,7 +155,8 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64_t ld, voi
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, int32_t c_dtype,
-                        int64_t ldc, float* c_amax, void* ws, size_t ws_bytes, void* stream) {
+                        int64_t ldc, float* c_amax, int64_t c_amax_cols, void* ws,
+                        size_t ws_bytes, void* stream) {
   nvfp4_status st = check_tensor(A);
   if (st != NVFP4_OK) return st;
   st = check_tensor(W);
@@ -169,6 +170,8 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (ldc < W->rows) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(C, 16) || ldc % 8 != 0) return NVFP4_ERR_MISALIGNED;
+  if (c_amax_cols < 0 || (c_amax_cols > 0 && (c_amax_cols % 256 != 0 || W->rows % c_amax_cols != 0)))
+    return NVFP4_ERR_INVALID_ARG;
   if (c_amax && !aligned(c_amax, 4)) return NVFP4_ERR_MISALIGNED;
   if (!ws || ws_bytes < kWsBytes) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;
@@ -188,6 +191,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
   g.c_dtype = c_dtype;
   g.ldc = ldc;
   g.c_amax = c_amax;
+  g.c_amax_cols = c_amax_cols;
   g.ws = ws;
   g.wait_limit_ns = g_wait_limit_ns.load();
   g.sm_count = dev.sm_count;
@@ -196,10 +200,12 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
 
 nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const void* k, const void* v,
                                   int64_t token_stride, const int32_t* dst_slots, int32_t n_frames,
-                                  void* ws, size_t ws_bytes, void* stream) {
+                                  float* k_amax_in, float* v_amax_in, void* ws, size_t ws_bytes,
+                                  void* stream) {
   nvfp4_status st = check_cache(cache);
   if (st != NVFP4_OK) return st;
   if (!k || !v || !dst_slots) return NVFP4_ERR_INVALID_ARG;
+  if ((k_amax_in == nullptr) != (v_amax_in == nullptr)) return NVFP4_ERR_INVALID_ARG;
   if (n_frames < 1 || n_frames > NVFP4_KV_MAX_CHUNK_FRAMES) return NVFP4_ERR_INVALID_ARG;
   const int64_t row_elems = int64_t(cache->heads) * cache->head_dim;
   if (token_stride < row_elems) return NVFP4_ERR_INVALID_ARG;
@@ -209,6 +215,8 @@ nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const void* k, co
       if (dst_slots[g] == dst_slots[f]) return NVFP4_ERR_INVALID_ARG;
   }
   if (!aligned(k, 16) || !aligned(v, 16) || token_stride % 8 != 0) return NVFP4_ERR_MISALIGNED;
+  if ((k_amax_in && !aligned(k_amax_in, 4)) || (v_amax_in && !aligned(v_amax_in, 4)))
+    return NVFP4_ERR_MISALIGNED;
   if (!ws || ws_bytes < kWsBytes) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;
   const DeviceInfo dev = current_device();
@@ -228,6 +236,8 @@ nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const void* k, co
   q.v_sf = cache->v_sf;
   q.k_st = cache->k_st;
   q.v_st = cache->v_st;
+  q.k_amax_in = k_amax_in;
+  q.v_amax_in = v_amax_in;
   q.ws = ws;
   q.sm_count = dev.sm_count;
   return cuda_status(launch_kv_quant(q, static_cast<cudaStream_t>(stream)));

@@ -322,6 +322,7 @@ struct Params {
   uint32_t tiles_m, tiles_n;
   uint32_t* status;
   uint32_t* c_amax;  // float bits of max|C| (atomicMax), or null
+  uint32_t amax_tiles;  // N tiles per c_amax word (0: one word)
   uint64_t wait_limit_ns;
   int32_t c_dtype;
 };
@@ -509,11 +510,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool bf16 = p.c_dtype == NVFP4_BF16;
     const uint32_t stage0 = sbase + kOffStage + ew * 2 * kStageBufBytes;
     uint32_t local = 0, nstore = 0;
-    // running max of |stored value| as magnitude bits: two bf16 halves, or fp32
-    uint32_t vmax = 0;
+    // running max of |stored value| as magnitude bits (two bf16 halves, or
+    // fp32) for c_amax word `word`; flushed when the tiles move to another word
+    uint32_t vmax = 0, word = 0;
     const bool want_max = p.c_amax != nullptr;
+    auto flush_max = [&]() {
+      // fold the bf16 halves into fp32 bits (bf16 bits << 16 is the same value)
+      const uint32_t bits = bf16 ? (max(vmax & 0xFFFFu, vmax >> 16) << 16) : vmax;
+      const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, bits);
+      if (lane == 0 && wmax != 0) atomicMax(p.c_amax + word, wmax);
+      vmax = 0;
+    };
     for (uint32_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
       const uint32_t tm = t % p.tiles_m, tn = t / p.tiles_m;
+      if (want_max && p.amax_tiles > 0 && tn / p.amax_tiles != word) {
+        flush_max();
+        word = tn / p.amax_tiles;
+      }
       // accumulator lanes past the last row of C hold zeros; leave them out anyway
       const bool row_live = want_max && tm * kBM + quad * 32 + uint32_t(lane) < p.M;
       const int32_t y = int32_t(tm * kBM + quad * 32);
@@ -572,12 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (want_max) {
-      // fold the bf16 halves into fp32 bits (bf16 bits << 16 is the same value)
-      const uint32_t bits = bf16 ? (max(vmax & 0xFFFFu, vmax >> 16) << 16) : vmax;
-      const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, bits);
-      if (lane == 0 && wmax != 0) atomicMax(p.c_amax, wmax);
-    }
+    if (want_max) flush_max();
     // drain: every store this warp issued has completed
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -674,6 +682,7 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.tiles_n = uint32_t(g.N / gemm::kBN);
   p.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(g.ws) + kWsStatus);
   p.c_amax = reinterpret_cast<uint32_t*>(g.c_amax);
+  p.amax_tiles = uint32_t(g.c_amax_cols / gemm::kBN);
   p.wait_limit_ns = g.wait_limit_ns;
   p.c_dtype = g.c_dtype;
   const uint32_t tiles = p.tiles_m * p.tiles_n;

@@ -43,6 +43,7 @@ struct LaunchKvQuant {
   const int32_t* slots;  // host, n_frames
   uint8_t *k_codes, *v_codes, *k_sf, *v_sf;
   float *k_st, *v_st;
+  float *k_amax_in, *v_amax_in;  // producer-accumulated amax per plane, or both NULL
   void* ws;
   int sm_count;
 };
@@ -70,7 +71,8 @@ struct LaunchGemm {
   void* c;
   int32_t c_dtype;
   int64_t ldc;
-  float* c_amax;  // max|C| accumulator, or NULL
+  float* c_amax;  // max|C| accumulator(s), or NULL
+  int64_t c_amax_cols;  // columns per accumulator word (0: one word)
   void* ws;
   uint64_t wait_limit_ns;
   int sm_count;

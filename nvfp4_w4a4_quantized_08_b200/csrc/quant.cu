@@ -442,6 +442,7 @@ struct KvQuantArgs {
   uint8_t* codes[2];   // slot pools
   uint8_t* sf[2];
   float* st[2];
+  float* amax_in[2];  // producer-accumulated amax per plane, or both null
   uint32_t* ws;
   uint32_t units_per_frame;
   FastDiv bpf_div;  // blocks per frame
@@ -469,7 +470,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4) kv_quant_kernel(KvQuantArgs 
     load_block<__nv_bfloat16>(block_ptr<__nv_bfloat16, kContig>(m, min(b, blocks - 1)),
                               cur[i]);
   }
-  if (threadIdx.x == 0) s_t_shared = take_scale(nullptr, nullptr, args.ws, plane);
+  if (threadIdx.x == 0)
+    s_t_shared = take_scale(nullptr, plane == 0 ? args.amax_in[0] : args.amax_in[1], args.ws, plane);
   __syncthreads();
   const float s_t = s_t_shared;
   const bool in_domain = tensor_scale_in_domain(s_t);
@@ -621,13 +623,16 @@ cudaError_t launch_kv_quant(const LaunchKvQuant& q, cudaStream_t st) {
   ka.codes[0] = q.k_codes; ka.codes[1] = q.v_codes;
   ka.sf[0] = q.k_sf; ka.sf[1] = q.v_sf;
   ka.st[0] = q.k_st; ka.st[1] = q.v_st;
+  ka.amax_in[0] = q.k_amax_in; ka.amax_in[1] = q.v_amax_in;
   ka.units_per_frame = uint32_t(int64_t(q.tpf) * row_elems / 8);
   ka.bpf_div = make_fastdiv(ka.units_per_frame / 2);
   for (int f = 0; f < NVFP4_KV_MAX_CHUNK_FRAMES; ++f) ka.slots[f] = f < q.n_frames ? q.slots[f] : 0;
   ka.n_frames = q.n_frames;
-  cudaError_t e = contig ? launch_amax<__nv_bfloat16, true>(aa, 2, q.sm_count, st)
-                         : launch_amax<__nv_bfloat16, false>(aa, 2, q.sm_count, st);
-  if (e != cudaSuccess) return e;
+  if (!q.k_amax_in) {
+    const cudaError_t e = contig ? launch_amax<__nv_bfloat16, true>(aa, 2, q.sm_count, st)
+                                 : launch_amax<__nv_bfloat16, false>(aa, 2, q.sm_count, st);
+    if (e != cudaSuccess) return e;
+  }
   return contig ? launch_kv_encode<true>(ka, q.sm_count, st)
                 : launch_kv_encode<false>(ka, q.sm_count, st);
 }

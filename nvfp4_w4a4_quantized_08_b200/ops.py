@@ -121,19 +121,26 @@ def dequantize(t: NVFP4Tensor, out: Optional[torch.Tensor] = None) -> torch.Tens
 
 def gemm(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype: torch.dtype = torch.bfloat16,
          out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-         c_amax: Optional[torch.Tensor] = None) -> torch.Tensor:
+         c_amax: Optional[torch.Tensor] = None, c_amax_cols: int = 0) -> torch.Tensor:
     """nvfp4_gemm: C = A W^T, [a.rows, w.rows] in bf16 or fp32.
 
-    c_amax: a one-element fp32 tensor that starts at 0 (or at a smaller running
-            max); the kernel raises it to max|C| over the values it stores.
+    c_amax: fp32 tensor that starts at 0 (or at a smaller running max); the
+            kernel raises it to max|C| over the values it stores.  With
+            c_amax_cols = 0 one element covers all of C; with c_amax_cols > 0
+            (a multiple of 256 dividing N) element g covers columns
+            [g * c_amax_cols, (g + 1) * c_amax_cols).
     """
+    if c_amax is not None:
+        need = 1 if c_amax_cols == 0 else max(1, w.rows // c_amax_cols)
+        if c_amax.dtype != torch.float32 or c_amax.numel() < need:
+            raise ValueError(f"c_amax needs {need} fp32 elements")
     if out is None:
         out = torch.empty(a.rows, w.rows, dtype=out_dtype, device=a.device)
     ws = workspace(a.device) if ws is None else ws
     sa, sw = a.c_struct(), w.c_struct()
     N.check(N.lib().nvfp4_gemm(ctypes.byref(sa), ctypes.byref(sw), out.data_ptr(),
-                               _dtype_code(out), out.stride(0), _ptr(c_amax), ws.data_ptr(),
-                               ws.numel(), _stream()), "nvfp4_gemm")
+                               _dtype_code(out), out.stride(0), _ptr(c_amax), c_amax_cols,
+                               ws.data_ptr(), ws.numel(), _stream()), "nvfp4_gemm")
     return out
 
 
@@ -157,9 +164,12 @@ class KVCache:
                          self.n_slots, self.tpf, self.heads, self.head_dim)
 
     def quant_chunk(self, k: torch.Tensor, v: torch.Tensor, dst_slots: Sequence[int],
-                    ws: Optional[torch.Tensor] = None) -> None:
+                    ws: Optional[torch.Tensor] = None, k_amax_in: Optional[torch.Tensor] = None,
+                    v_amax_in: Optional[torch.Tensor] = None) -> None:
         """nvfp4_kv_quant_chunk.  k, v: bf16 views [tokens, heads*head_dim] (or
-        [tokens, heads, head_dim]) with unit stride inside a token."""
+        [tokens, heads, head_dim]) with unit stride inside a token.
+        k_amax_in, v_amax_in: both None (amax pass), or one-element fp32
+        tensors holding max|K|, max|V| from the producer; reset to 0."""
         token_stride = k.stride(0)
         if v.stride(0) != token_stride:
             raise ValueError("k and v must share a token stride")
@@ -167,8 +177,9 @@ class KVCache:
         ws = workspace(k.device) if ws is None else ws
         cs = self.c_struct()
         N.check(N.lib().nvfp4_kv_quant_chunk(ctypes.byref(cs), k.data_ptr(), v.data_ptr(),
-                                             token_stride, slots, len(dst_slots), ws.data_ptr(),
-                                             ws.numel(), _stream()), "nvfp4_kv_quant_chunk")
+                                             token_stride, slots, len(dst_slots), _ptr(k_amax_in),
+                                             _ptr(v_amax_in), ws.data_ptr(), ws.numel(),
+                                             _stream()), "nvfp4_kv_quant_chunk")
 
     def dequant_window(self, slot_ids: Sequence[int], k_out: Optional[torch.Tensor] = None,
                        v_out: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:

@@ -89,7 +89,7 @@ def test_gemm_rejects(L):
     a = _tensor(rows=2640, cols=3072)
     w = _tensor(rows=9216, cols=3072)
     g = L.nvfp4_gemm
-    ok_args = (FAKE, N.BF16, 9216, None, FAKE, 256, None)
+    ok_args = (FAKE, N.BF16, 9216, None, 0, FAKE, 256, None)
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9216, cols=3072, layout=N.SF_ROWMAJOR)),
              *ok_args) == N.ERR_INVALID_ARG
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9216, cols=2048)),
@@ -97,17 +97,20 @@ def test_gemm_rejects(L):
     assert g(ctypes.byref(_tensor(rows=2640, cols=3056)),
              ctypes.byref(_tensor(rows=9216, cols=3056)), *ok_args) == N.ERR_UNSUPPORTED_SHAPE
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9200, cols=3072)),
-             FAKE, N.BF16, 9216, None, FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # N % 256
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9000, None, FAKE, 256,
+             FAKE, N.BF16, 9216, None, 0, FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # N % 256
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9000, None, 0, FAKE, 256,
              None) == N.ERR_INVALID_ARG  # ldc < N
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9220, None, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9220, None, 0, FAKE, 256,
              None) == N.ERR_MISALIGNED
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, 5, 9216, None, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, 5, 9216, None, 0, FAKE, 256,
              None) == N.ERR_INVALID_ARG
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, None, FAKE, 4,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, None, 0, FAKE, 4,
              None) == N.ERR_WORKSPACE
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, FAKE + 1, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, FAKE + 1, 0, FAKE, 256,
              None) == N.ERR_MISALIGNED  # c_amax
+    for cols in (-256, 100, 2048, 9216 * 2):  # not a multiple of 256 dividing N
+        assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, FAKE, cols, FAKE, 256,
+                 None) == N.ERR_INVALID_ARG
 
 
 def _cache(n_slots=12, tpf=880, heads=24, hd=128):
@@ -119,18 +122,29 @@ def test_kv_rejects(L):
     q = L.nvfp4_kv_quant_chunk
     S = ctypes.c_int32 * 9
     slots = S(0, 1, 2, 3, 4, 5, 6, 7, 8)
-    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 9, FAKE, 256, None) == N.ERR_INVALID_ARG
-    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 0, FAKE, 256, None) == N.ERR_INVALID_ARG
+    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 9, None, None, FAKE, 256,
+             None) == N.ERR_INVALID_ARG
+    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 0, None, None, FAKE, 256,
+             None) == N.ERR_INVALID_ARG
     bad = (ctypes.c_int32 * 2)(0, 12)
-    assert q(ctypes.byref(c), FAKE, FAKE, 3072, bad, 2, FAKE, 256, None) == N.ERR_INVALID_ARG
+    assert q(ctypes.byref(c), FAKE, FAKE, 3072, bad, 2, None, None, FAKE, 256,
+             None) == N.ERR_INVALID_ARG
     rep = (ctypes.c_int32 * 2)(3, 3)
-    assert q(ctypes.byref(c), FAKE, FAKE, 3072, rep, 2, FAKE, 256, None) == N.ERR_INVALID_ARG
-    assert q(ctypes.byref(c), FAKE, FAKE, 3000, slots, 2, FAKE, 256,
+    assert q(ctypes.byref(c), FAKE, FAKE, 3072, rep, 2, None, None, FAKE, 256,
+             None) == N.ERR_INVALID_ARG
+    assert q(ctypes.byref(c), FAKE, FAKE, 3000, slots, 2, None, None, FAKE, 256,
              None) == N.ERR_INVALID_ARG  # token stride < heads * head_dim
-    assert q(ctypes.byref(c), FAKE, FAKE, 3076, slots, 2, FAKE, 256, None) == N.ERR_MISALIGNED
-    assert q(ctypes.byref(_cache(hd=40)), FAKE, FAKE, 3072, slots, 2, FAKE, 256,
+    assert q(ctypes.byref(c), FAKE, FAKE, 3076, slots, 2, None, None, FAKE, 256,
+             None) == N.ERR_MISALIGNED
+    assert q(ctypes.byref(_cache(hd=40)), FAKE, FAKE, 3072, slots, 2, None, None, FAKE, 256,
              None) == N.ERR_UNSUPPORTED_SHAPE
-    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 2, FAKE, 16, None) == N.ERR_WORKSPACE
+    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 2, None, None, FAKE, 16,
+             None) == N.ERR_WORKSPACE
+    # the producer's amax words come as a pair or not at all
+    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 2, FAKE, None, FAKE, 256,
+             None) == N.ERR_INVALID_ARG
+    assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 2, FAKE, FAKE + 2, FAKE, 256,
+             None) == N.ERR_MISALIGNED
     d = L.nvfp4_kv_dequant_window
     ids = (ctypes.c_int32 * 3)(0, 5, 12)
     assert d(ctypes.byref(c), ids, 3, FAKE, FAKE, None) == N.ERR_INVALID_ARG

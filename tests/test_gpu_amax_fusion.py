@@ -103,3 +103,39 @@ def test_amax_in_out_of_domain_is_reported_and_reset():
     assert zero.s_t.item() == 0.0 and not zero.codes.any()
     assert nv.device_status() == 0
     assert np.isfinite(word.item())
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_c_amax_per_column_group(out_dtype):
+    """c_amax_cols = 256, 512, N: word g is max|C| over its own columns only."""
+    qa, qw = _operands(300, 1536, 512, seed=31)
+    for cols in (256, 512, 1536):
+        words = torch.zeros(1536 // cols, dtype=torch.float32, device="cuda")
+        y = nv.gemm(qa, qw, out_dtype=out_dtype, c_amax=words, c_amax_cols=cols)
+        torch.cuda.synchronize()
+        ref = y.float().abs().reshape(300, 1536 // cols, cols).amax(dim=(0, 2))
+        assert torch.equal(words, ref), (cols, words, ref)
+
+
+def test_kv_chunk_from_qkv_gemm_amax(orc):
+    """QKV projection with one amax word per Q/K/V third; the K and V words
+    feed kv_quant_chunk, which then writes the same bytes as with its own
+    amax pass, and leaves both words at 0."""
+    tpf, heads, hd = 16, 4, 64
+    d = heads * hd
+    qa, qw = _operands(3 * tpf, 3 * d, 256, seed=41)
+    words = torch.zeros(3, dtype=torch.float32, device="cuda")
+    qkv = nv.gemm(qa, qw, out_dtype=torch.bfloat16, c_amax=words, c_amax_cols=d)
+    torch.cuda.synchronize()
+    assert words[1].item() == qkv[:, d:2 * d].float().abs().max().item()
+    assert words[2].item() == qkv[:, 2 * d:].float().abs().max().item()
+    fused = nv.KVCache(4, tpf, heads, hd)
+    plain = nv.KVCache(4, tpf, heads, hd)
+    fused.quant_chunk(qkv[:, d:2 * d], qkv[:, 2 * d:], [3, 0, 2], k_amax_in=words[1:2],
+                      v_amax_in=words[2:3])
+    plain.quant_chunk(qkv[:, d:2 * d], qkv[:, 2 * d:], [3, 0, 2])
+    torch.cuda.synchronize()
+    assert words[1].item() == 0.0 and words[2].item() == 0.0
+    for name in ("k_codes", "v_codes", "k_sf", "v_sf", "k_st", "v_st"):
+        assert torch.equal(getattr(fused, name), getattr(plain, name)), name
+    assert nv.device_status() == 0
