@@ -86,7 +86,9 @@ def lib() -> ctypes.CDLL:
         L.orc_gemm.restype = i32
         L.orc_gemm.argtypes = [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, i64, vp, vp]
         L.orc_kv_quant_chunk.restype = i32
-        L.orc_kv_quant_chunk.argtypes = [vp, i64, i32, i32, i32, i32, vp, vp, vp]
+        L.orc_kv_quant_chunk.argtypes = [vp, i64, i32, i32, i32, i32, vp, vp, vp, i32]
+        L.orc_block_scale_rule.restype = i32
+        L.orc_block_scale_rule.argtypes = [vp, ctypes.c_float, i32]
         L.orc_kv_dequant_window.restype = i32
         L.orc_kv_dequant_window.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, vp]
         L.orc_set_threads.restype = i32
@@ -245,10 +247,11 @@ def gemm(a: Tuple[np.ndarray, np.ndarray, float], w: Tuple[np.ndarray, np.ndarra
 
 
 def kv_quant_chunk(kv: np.ndarray, n_frames: int, tpf: int, heads: int, head_dim: int,
-                   token_stride: Optional[int] = None
+                   token_stride: Optional[int] = None, rule: int = 0
                    ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """kv: bf16 bits, flat buffer holding n_frames*tpf tokens at token_stride
-    elements apart.  -> (codes [n_frames, tpf*heads*head_dim/2],
+    elements apart.  rule 0: block max onto 6; rule 1: Four Over Six.
+    -> (codes [n_frames, tpf*heads*head_dim/2],
     sf [n_frames, tpf*heads*head_dim/16], s_t [n_frames])."""
     kv = np.ascontiguousarray(kv, np.uint16)
     ts = heads * head_dim if token_stride is None else token_stride
@@ -257,9 +260,18 @@ def kv_quant_chunk(kv: np.ndarray, n_frames: int, tpf: int, heads: int, head_dim
     sf = np.empty((n_frames, per // 16), np.uint8)
     st = np.empty(n_frames, np.float32)
     rc = lib().orc_kv_quant_chunk(_ptr(kv), ts, n_frames, tpf, heads, head_dim, _ptr(codes),
-                                  _ptr(sf), _ptr(st))
+                                  _ptr(sf), _ptr(st), rule)
     _check(rc, "kv_quant_chunk")
     return codes, sf, st
+
+
+def block_scale_rule(block: np.ndarray, s_t: float, rule: int) -> int:
+    """Scale byte of one 16-element fp32 block under `rule` (0: onto 6,
+    1: Four Over Six)."""
+    block = np.ascontiguousarray(block, np.float32)
+    if block.size != 16:
+        raise ValueError("a block has 16 elements")
+    return int(lib().orc_block_scale_rule(_ptr(block), float(s_t), int(rule)))
 
 
 def kv_dequant_window(pool_codes: np.ndarray, pool_sf: np.ndarray, pool_st: np.ndarray,

@@ -32,6 +32,13 @@
  * value set in binary64.  GEMM references are binary64 sums of exactly
  * dequantized operands.
  *
+ * KV scale rule "Four Over Six" (tailorednewshub.com article, section
+ * "Inferencia W4A4 NVFP4": the KV cache uses micro-block scaling with an
+ * adaptive scale choice named Four Over Six; the pages give no formula).  The
+ * reading taken here: per 16-element block, scale the block maximum onto 6
+ * (the standard rule) or onto 4, quantize with each, and keep the one whose
+ * squared error against the exactly decoded values is smaller (ties keep 6).
+ *
  * Parity pins (tests/test_oracle_*.py): exhaustive decode of all 16 E2M1 codes
  * and 256 E4M3 bytes against ml_dtypes / torch, encode against the same
  * libraries on tie and random values, exact round trips of representable
@@ -230,13 +237,50 @@ int orc_element_code(float x, int s_b_byte, float s_t) {
   return orc_e2m1_encode(y);
 }
 
+/* Block scale with the block maximum mapped onto `top` (6: the standard
+ * rule; 4: the Four Over Six alternative): E4M3_RNE_sat(amax_b / (top * s_t)),
+ * the product rounded first. */
+static int block_scale_onto(float amax_b, float s_t, float top) {
+  if (s_t == 0.0f) return 0;
+  float t_st = top * s_t;
+  float r = amax_b / t_st;
+  return orc_e4m3_encode(r);
+}
+
+/* Squared error of a 16-element block coded with scale byte s_b, against the
+ * exactly decoded values v(q) * s_b * s_t (exact in binary64): the sum, in
+ * element order, of (|x_i| - v(|q_i|) * s_b * s_t)^2, each operation one
+ * binary64 rounding. */
+static double block_sq_error(const float* xs, int s_b, float s_t) {
+  double e = 0.0;
+  for (int t = 0; t < 16; ++t) {
+    int q = orc_element_code(xs[t], s_b, s_t);
+    double recon = orc_e2m1_value(q & 7) * orc_e4m3_value(s_b);
+    recon = recon * (double)s_t;
+    double diff = (double)fabsf(xs[t]) - recon;
+    e = e + diff * diff;
+  }
+  return e;
+}
+
+/* Scale byte of a block under `rule` (0: onto 6; 1: Four Over Six). */
+int orc_block_scale_rule(const float* xs, float s_t, int rule) {
+  float amax_b = 0.0f;
+  for (int t = 0; t < 16; ++t) amax_b = fmaxf(amax_b, fabsf(xs[t]));
+  int s6 = block_scale_onto(amax_b, s_t, 6.0f);
+  if (rule == 0) return s6;
+  int s4 = block_scale_onto(amax_b, s_t, 4.0f);
+  return block_sq_error(xs, s4, s_t) < block_sq_error(xs, s6, s_t) ? s4 : s6;
+}
+
 /* Quantize a rows x cols tensor (row stride ld elements) to NVFP4.
  *   codes: [rows][cols/2] bytes, element 2j in the low nibble of byte j
  *   sf:    [rows][cols/16] E4M3 bytes (row-major)
  *   s_t:   tensor scale (computed, or taken from *s_t_in when non-NULL)
  */
-int orc_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
-                 uint8_t* codes, uint8_t* sf, float* s_t_out, const float* s_t_in) {
+static int quantize_rule(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                         uint8_t* codes, uint8_t* sf, float* s_t_out, const float* s_t_in,
+                         int rule) {
   if (cols % 16 != 0 || rows < 0 || ld < cols || (dtype != 0 && dtype != 1)) return ORC_ERR_ARG;
   float s_t;
   if (s_t_in) {
@@ -258,7 +302,7 @@ int orc_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
         if (!isfinite(xs[t])) bad = 1;
         amax_b = fmaxf(amax_b, fabsf(xs[t]));
       }
-      int s_b = orc_block_scale(amax_b, s_t);
+      int s_b = rule == 0 ? orc_block_scale(amax_b, s_t) : orc_block_scale_rule(xs, s_t, rule);
       sf[i * nkb + kb] = (uint8_t)s_b;
       for (int t = 0; t < 16; t += 2) {
         int q0 = orc_element_code(xs[t], s_b, s_t);
@@ -270,6 +314,11 @@ int orc_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
   if (bad) return ORC_ERR_NONFINITE;
   *s_t_out = s_t;
   return ORC_OK;
+}
+
+int orc_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                 uint8_t* codes, uint8_t* sf, float* s_t_out, const float* s_t_in) {
+  return quantize_rule(x, dtype, rows, cols, ld, codes, sf, s_t_out, s_t_in, 0);
 }
 
 /* ------------------------------------------------------------------ */
@@ -380,9 +429,9 @@ int orc_gemm(const uint8_t* a_codes, const uint8_t* a_sf, float a_st, const uint
  * to codes + f*frame_code_bytes and sf + f*frame_sf_bytes (row-major
  * [tpf][heads][head_dim/16]); its tensor scale to s_t[f]. */
 int orc_kv_quant_chunk(const uint16_t* kv, int64_t token_stride, int n_frames, int tpf, int heads,
-                       int head_dim, uint8_t* codes, uint8_t* sf, float* s_t) {
+                       int head_dim, uint8_t* codes, uint8_t* sf, float* s_t, int rule) {
   if (head_dim % 16 != 0 || n_frames < 0 || tpf < 0 || heads < 0 ||
-      token_stride < (int64_t)heads * head_dim)
+      token_stride < (int64_t)heads * head_dim || (rule != 0 && rule != 1))
     return ORC_ERR_ARG;
   int64_t tokens = (int64_t)n_frames * tpf;
   int64_t row_elems = (int64_t)heads * head_dim;
@@ -393,7 +442,7 @@ int orc_kv_quant_chunk(const uint16_t* kv, int64_t token_stride, int n_frames, i
   for (int64_t t = 0; t < tokens; ++t)
     memcpy(dense + t * row_elems, kv + t * token_stride, sizeof(uint16_t) * (size_t)row_elems);
   float st;
-  int rc = orc_quantize(dense, 0, tokens * heads, head_dim, head_dim, codes, sf, &st, NULL);
+  int rc = quantize_rule(dense, 0, tokens * heads, head_dim, head_dim, codes, sf, &st, NULL, rule);
   free(dense);
   if (rc) return rc;
   for (int f = 0; f < n_frames; ++f) s_t[f] = st;
