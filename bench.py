@@ -345,6 +345,34 @@ def config_block(args):
                          "GELU not run (outside the NVFP4 path)"}
 
 
+def time_kv_four_over_six(step: "Step", dev, reps: int = 20) -> float:
+    """Device ms of one nvfp4_kv_quant_chunk (3 frames of K and V read from a
+    QKV output, amax pass included) with the Four Over Six scale rule."""
+    cache = nv.KVCache(POOL, TPF, wl.HEADS, wl.HEAD_DIM, device=dev,
+                       scale_rule=nv.SCALE_FOUR_OVER_SIX)
+    k, v = step.qkv_out[:, D:2 * D], step.qkv_out[:, 2 * D:]
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            cache.quant_chunk(k, v, step.new_slots, ws=nv.workspace(dev))
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):
+                cache.quant_chunk(k, v, step.new_slots, ws=nv.workspace(dev))
+    torch.cuda.current_stream(dev).wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    del g
+    return e0.elapsed_time(e1) / reps
+
+
 def run_ours(args):
     world = env_int("WORLD_SIZE", 1)
     rank = env_int("RANK", 0)
@@ -446,6 +474,9 @@ def run_ours(args):
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     e2e_value = job_throughput(flops_step, world, ms_e2e / args.steps)
     status = nv.device_status(step.ws)
+    # the KV chunk under Four Over Six (the adaptive KV scale rule; not on the
+    # step's path): one layer's 3 new frames of K and V, graph-replayed
+    fos_ms = time_kv_four_over_six(step, dev)
 
     peaks, peak_src = measured_peaks()
     fp4_peak = 4.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -482,6 +513,11 @@ def run_ours(args):
                          "frac_hbm": kv_bytes / (kv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "hbm_peak_gbs": peaks["hbm_gbs"]},
             "codec": codec,
+            "kv_quant_four_over_six": {
+                "us": fos_ms * 1e3,
+                "gb_s": CODEC_BYTES["kv_quant"] / (fos_ms * 1e-3) / 1e9,
+                "frac_hbm": CODEC_BYTES["kv_quant"] / (fos_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "vs_onto_6_us": kernel_ms["kv_quant"] / args.layers * 1e3},
             "gemm": {"tflops": gemm_tflops, "ms_per_step": gemm_ms,
                      "launches_per_step": gemm_launches,
                      "by_shape_ms": {k: v for k, v in kernel_ms.items() if k.startswith("gemm")}},

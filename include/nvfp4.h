@@ -80,6 +80,16 @@ typedef enum { NVFP4_BF16 = 0, NVFP4_FP32 = 1 } nvfp4_dtype;
  *     nvfp4_gemm operands must use this layout. */
 typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA128x4 = 1 } nvfp4_sf_layout;
 
+/* How a KV chunk's block scales are chosen.
+ *   ONTO_6: s_b = E4M3_RNE_sat(amax_b / (6 s_t)), the recipe of nvfp4_quantize.
+ *   FOUR_OVER_SIX: the adaptive choice the pages name for the KV cache
+ *     (tailorednewshub.com LongLive-2.0 article, section "Inferencia W4A4
+ *     NVFP4"), read as: per block, the scale with the block maximum onto 6 or
+ *     onto 4 (E4M3_RNE_sat(amax_b / (4 s_t))), whichever codes the block with
+ *     the smaller squared error against the exactly decoded values (binary64,
+ *     element order; 6 on a tie).  The stored format is unchanged. */
+typedef enum { NVFP4_SCALE_ONTO_6 = 0, NVFP4_SCALE_FOUR_OVER_SIX = 1 } nvfp4_scale_rule;
+
 /* An NVFP4 tensor of rows x cols elements (cols a multiple of 16).
  *   codes: device, [rows][cols/2] bytes; element 2j in the low nibble of
  *          byte j, element 2j+1 in the high nibble; sign in bit 3 of a nibble.
@@ -103,6 +113,7 @@ typedef struct {
  *                     row-major ([token][head][head_dim/16]) E4M3 scales
  *   k_st, v_st:       device, [n_slots] floats: the tensor scale of the chunk
  *                     that last wrote the slot
+ *   scale_rule:       nvfp4_scale_rule used by nvfp4_kv_quant_chunk
  * Code and scale pools must be 16-byte aligned; head_dim a multiple of 16. */
 typedef struct {
   uint8_t* k_codes;
@@ -115,6 +126,7 @@ typedef struct {
   int32_t tokens_per_frame;
   int32_t heads;
   int32_t head_dim;
+  int32_t scale_rule; /* nvfp4_scale_rule */
 } nvfp4_kv_cache;
 
 /* Most frames one kv_quant_chunk call writes (the pages' 8-frame block) and

@@ -27,6 +27,8 @@ BF16 = 0
 FP32 = 1
 SF_ROWMAJOR = 0
 SF_MMA128x4 = 1
+SCALE_ONTO_6 = 0
+SCALE_FOUR_OVER_SIX = 1
 KV_MAX_CHUNK_FRAMES = 8
 KV_MAX_WINDOW_SLOTS = 256
 
@@ -48,7 +50,8 @@ class KvCache(ctypes.Structure):
                 ("k_sf", ctypes.c_void_p), ("v_sf", ctypes.c_void_p),
                 ("k_st", ctypes.c_void_p), ("v_st", ctypes.c_void_p),
                 ("n_slots", ctypes.c_int32), ("tokens_per_frame", ctypes.c_int32),
-                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("scale_rule", ctypes.c_int32)]
 
 
 class NVFP4Error(RuntimeError):

@@ -56,6 +56,8 @@ nvfp4_status check_cache(const nvfp4_kv_cache* c) {
     return NVFP4_ERR_INVALID_ARG;
   if (c->n_slots <= 0 || c->tokens_per_frame <= 0 || c->heads <= 0 || c->head_dim <= 0)
     return NVFP4_ERR_INVALID_ARG;
+  if (c->scale_rule != NVFP4_SCALE_ONTO_6 && c->scale_rule != NVFP4_SCALE_FOUR_OVER_SIX)
+    return NVFP4_ERR_INVALID_ARG;
   if (c->head_dim % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const int64_t per_frame = int64_t(c->tokens_per_frame) * c->heads * c->head_dim;
   if (per_frame * c->n_slots / 8 >= (int64_t(1) << 32)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -238,6 +240,7 @@ nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const void* k, co
   q.v_st = cache->v_st;
   q.k_amax_in = k_amax_in;
   q.v_amax_in = v_amax_in;
+  q.scale_rule = cache->scale_rule;
   q.ws = ws;
   q.sm_count = dev.sm_count;
   return cuda_status(launch_kv_quant(q, static_cast<cudaStream_t>(stream)));

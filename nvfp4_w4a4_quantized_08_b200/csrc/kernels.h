@@ -44,6 +44,7 @@ struct LaunchKvQuant {
   uint8_t *k_codes, *v_codes, *k_sf, *v_sf;
   float *k_st, *v_st;
   float *k_amax_in, *v_amax_in;  // producer-accumulated amax per plane, or both NULL
+  int32_t scale_rule;            // nvfp4_scale_rule
   void* ws;
   int sm_count;
 };

@@ -180,11 +180,13 @@ struct ScaleConsts {
   bool zero;
 };
 
-__device__ __forceinline__ ScaleConsts make_consts(float s_t) {
+// Constants of the block-scale division amax_b / (top * s_t); top = 6 is the
+// recipe, 4 the Four Over Six alternative.
+__device__ __forceinline__ ScaleConsts make_consts(float s_t, float top = 6.0f) {
   ScaleConsts k;
   k.s_t = s_t;
   k.zero = (s_t == 0.0f);
-  k.c = __fmul_rn(6.0f, s_t);
+  k.c = __fmul_rn(top, s_t);
   float rc = k.zero ? 0.0f : __frcp_rn(k.c);
   k.rc_lo = __fmul_rn(rc, 1.0f - 0x1p-20f);
   k.rc_hi = __fmul_rn(rc, 1.0f + 0x1p-20f);
@@ -359,6 +361,54 @@ __device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, con
   return sb;
 }
 
+// ---- Four Over Six (KV chunks)
+// Magnitude of E2M1 code q (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ double e2m1_magnitude(uint32_t q) {
+  const double m = (q & 1) ? 1.5 : 1.0;
+  return q < 2 ? 0.5 * double(q) : ldexp(m, int(q >> 1) - 1);
+}
+
+// Squared error of a block coded as (sb, codes) against the exactly decoded
+// values: sum over the 16 elements, in order, of (|x| - v(|q|) * s_b * s_t)^2,
+// each operation one binary64 rounding (explicit intrinsics: no contraction).
+template <typename InT>
+__device__ __forceinline__ double block_sq_error(const RawBlock<InT>& raw, uint2 codes,
+                                                 uint32_t sb, float s_t) {
+  float a[16];
+  unit_values<InT>(raw.h[0], a);
+  unit_values<InT>(raw.h[1], a + 8);
+  const double sbv = double(e4m3_to_f32(sb & 0x7Fu));
+  double e = 0.0;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    const uint32_t q = ((t < 8 ? codes.x : codes.y) >> (4 * (t & 7))) & 7u;
+    double recon = __dmul_rn(e2m1_magnitude(q), sbv);
+    recon = __dmul_rn(recon, double(s_t));
+    const double diff = __dsub_rn(double(fabsf(a[t])), recon);
+    e = __dadd_rn(e, __dmul_rn(diff, diff));
+  }
+  return e;
+}
+
+// A block under Four Over Six: coded both ways (maximum onto 6 with k6, onto
+// 4 with k4), the one with the smaller squared error kept, 6 on a tie.
+template <typename InT>
+__device__ __forceinline__ uint32_t quantize_block_4over6(const RawBlock<InT>& raw,
+                                                          const float* inv_tab,
+                                                          const ScaleConsts& k6,
+                                                          const ScaleConsts& k4, uint2& codes) {
+  uint2 c6, c4;
+  const uint32_t sb6 = quantize_block<InT>(raw, inv_tab, k6, c6);
+  const uint32_t sb4 = quantize_block<InT>(raw, inv_tab, k4, c4);
+  codes = c6;
+  if (sb4 == sb6) return sb6;
+  if (block_sq_error<InT>(raw, c4, sb4, k6.s_t) < block_sq_error<InT>(raw, c6, sb6, k6.s_t)) {
+    codes = c4;
+    return sb4;
+  }
+  return sb6;
+}
+
 // The dense quantizer.  Each thread encodes whole blocks (grid-stride over
 // the tensor's blocks), loading the blocks of its next pass before it encodes
 // the ones it holds; the first loads go out before the tensor scale is known.
@@ -450,8 +500,9 @@ struct KvQuantArgs {
   int32_t n_frames;
 };
 
-template <bool kContig>
-__global__ void __launch_bounds__(kQuantThreads, 4) kv_quant_kernel(KvQuantArgs args) {
+template <bool kContig, int kRule>
+__global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4 : 2)
+    kv_quant_kernel(KvQuantArgs args) {
   constexpr int D = Prefetch<__nv_bfloat16>::kDepth;
   __shared__ float inv_tab[128];
   __shared__ float s_t_shared;
@@ -483,6 +534,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) kv_quant_kernel(KvQuantArgs 
     uint8_t* const codes_pool = plane == 0 ? args.codes[0] : args.codes[1];
     uint8_t* const sf_pool = plane == 0 ? args.sf[0] : args.sf[1];
     const ScaleConsts k = make_consts(s_t);
+    const ScaleConsts k4 = make_consts(s_t, 4.0f);
     const uint32_t bpf = args.units_per_frame >> 1;  // blocks per frame
     for (; b0 < blocks; b0 += D * stride) {
       RawBlock<__nv_bfloat16> nxt[D];
@@ -497,7 +549,10 @@ __global__ void __launch_bounds__(kQuantThreads, 4) kv_quant_kernel(KvQuantArgs 
         const uint32_t b = b0 + i * stride;
         if (b < blocks) {
           uint2 codes;
-          const uint32_t sb = quantize_block<__nv_bfloat16>(cur[i], inv_tab, k, codes);
+          const uint32_t sb =
+              kRule == NVFP4_SCALE_ONTO_6
+                  ? quantize_block<__nv_bfloat16>(cur[i], inv_tab, k, codes)
+                  : quantize_block_4over6<__nv_bfloat16>(cur[i], inv_tab, k, k4, codes);
           const uint32_t f = fast_div(args.bpf_div, b);
           const uint32_t bf = b - f * bpf;
           const size_t slot = size_t(args.slots[f]);
@@ -548,11 +603,12 @@ static cudaError_t launch_encode(const QuantArgs& a, int sm_count, cudaStream_t 
                     a);
 }
 
-template <bool kContig>
+template <bool kContig, int kRule>
 static cudaError_t launch_kv_encode(const KvQuantArgs& a, int sm_count, cudaStream_t st) {
-  static const int per_sm = resident_per_sm(kv_quant_kernel<kContig>);
+  static const int per_sm = resident_per_sm(kv_quant_kernel<kContig, kRule>);
   const int grid = wave_grid(a.in[0].units, 1, per_sm, sm_count, 2);
-  return launch_pdl(kv_quant_kernel<kContig>, dim3(grid, 2), dim3(kQuantThreads), 0, st, a);
+  return launch_pdl(kv_quant_kernel<kContig, kRule>, dim3(grid, 2), dim3(kQuantThreads), 0, st,
+                    a);
 }
 
 static InMap make_inmap(const void* x, int64_t rows_total, int64_t cols, int64_t rows_per_group,
@@ -633,8 +689,11 @@ cudaError_t launch_kv_quant(const LaunchKvQuant& q, cudaStream_t st) {
                                  : launch_amax<__nv_bfloat16, false>(aa, 2, q.sm_count, st);
     if (e != cudaSuccess) return e;
   }
-  return contig ? launch_kv_encode<true>(ka, q.sm_count, st)
-                : launch_kv_encode<false>(ka, q.sm_count, st);
+  if (q.scale_rule == NVFP4_SCALE_FOUR_OVER_SIX)
+    return contig ? launch_kv_encode<true, NVFP4_SCALE_FOUR_OVER_SIX>(ka, q.sm_count, st)
+                  : launch_kv_encode<false, NVFP4_SCALE_FOUR_OVER_SIX>(ka, q.sm_count, st);
+  return contig ? launch_kv_encode<true, NVFP4_SCALE_ONTO_6>(ka, q.sm_count, st)
+                : launch_kv_encode<false, NVFP4_SCALE_ONTO_6>(ka, q.sm_count, st);
 }
 
 }  // namespace nvfp4

@@ -148,8 +148,10 @@ class KVCache:
     """The NVFP4 KV cache of one layer: n_slots frame slots for K and V."""
 
     def __init__(self, n_slots: int, tokens_per_frame: int, heads: int, head_dim: int,
-                 device="cuda"):
+                 device="cuda", scale_rule: int = N.SCALE_ONTO_6):
+        """scale_rule: N.SCALE_ONTO_6 (the recipe) or N.SCALE_FOUR_OVER_SIX."""
         per = tokens_per_frame * heads * head_dim
+        self.scale_rule = scale_rule
         self.n_slots, self.tpf, self.heads, self.head_dim = n_slots, tokens_per_frame, heads, head_dim
         self.k_codes = torch.zeros(n_slots, per // 2, dtype=torch.uint8, device=device)
         self.v_codes = torch.zeros_like(self.k_codes)
@@ -161,7 +163,7 @@ class KVCache:
     def c_struct(self) -> N.KvCache:
         return N.KvCache(self.k_codes.data_ptr(), self.v_codes.data_ptr(), self.k_sf.data_ptr(),
                          self.v_sf.data_ptr(), self.k_st.data_ptr(), self.v_st.data_ptr(),
-                         self.n_slots, self.tpf, self.heads, self.head_dim)
+                         self.n_slots, self.tpf, self.heads, self.head_dim, self.scale_rule)
 
     def quant_chunk(self, k: torch.Tensor, v: torch.Tensor, dst_slots: Sequence[int],
                     ws: Optional[torch.Tensor] = None, k_amax_in: Optional[torch.Tensor] = None,

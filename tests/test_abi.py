@@ -113,8 +113,8 @@ def test_gemm_rejects(L):
                  None) == N.ERR_INVALID_ARG
 
 
-def _cache(n_slots=12, tpf=880, heads=24, hd=128):
-    return N.KvCache(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, n_slots, tpf, heads, hd)
+def _cache(n_slots=12, tpf=880, heads=24, hd=128, rule=0):
+    return N.KvCache(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, n_slots, tpf, heads, hd, rule)
 
 
 def test_kv_rejects(L):
@@ -140,6 +140,9 @@ def test_kv_rejects(L):
              None) == N.ERR_UNSUPPORTED_SHAPE
     assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 2, None, None, FAKE, 16,
              None) == N.ERR_WORKSPACE
+    # scale rules: 0 (onto 6) and 1 (Four Over Six) only
+    assert q(ctypes.byref(_cache(rule=2)), FAKE, FAKE, 3072, slots, 2, None, None, FAKE, 256,
+             None) == N.ERR_INVALID_ARG
     # the producer's amax words come as a pair or not at all
     assert q(ctypes.byref(c), FAKE, FAKE, 3072, slots, 2, FAKE, None, FAKE, 256,
              None) == N.ERR_INVALID_ARG

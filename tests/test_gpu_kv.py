@@ -117,3 +117,35 @@ def test_bad_slots_rejected_on_host():
         cache.quant_chunk(k, k, [1, 1])  # repeated
     with pytest.raises(nv.NVFP4Error):
         cache.dequant_window([0, -1])
+
+
+@pytest.mark.parametrize("token_stride_extra", [0, 64])
+def test_four_over_six_chunk_matches_oracle(orc, token_stride_extra):
+    """Four Over Six chunks: codes, scales and s_t byte-identical to the
+    oracle's rule, some block scales different from the onto-6 rule, and the
+    window rebuild of those slots identical to the oracle's."""
+    tpf, heads, hd, nf = 40, 6, 64, 3
+    g = torch.Generator().manual_seed(23)
+    sig = torch.tensor([0.5, 1.0, 2.0, 3.0, 4.0, 0.7]).view(1, heads, 1)
+    kv = (torch.randn(nf * tpf, heads, hd, generator=g) * sig).to(torch.bfloat16)
+    width = heads * hd + token_stride_extra
+    buf = torch.zeros(nf * tpf, width, dtype=torch.bfloat16)
+    buf[:, :heads * hd] = kv.reshape(nf * tpf, -1)
+    cache = nv.KVCache(5, tpf, heads, hd, scale_rule=nv.SCALE_FOUR_OVER_SIX)
+    d = buf.cuda()
+    cache.quant_chunk(d[:, :heads * hd], d[:, :heads * hd], [4, 1, 2])
+    bits_flat = bits(buf).reshape(-1)
+    codes, sf, st = orc.kv_quant_chunk(bits_flat, nf, tpf, heads, hd, token_stride=width, rule=1)
+    _, sf6, _ = orc.kv_quant_chunk(bits_flat, nf, tpf, heads, hd, token_stride=width, rule=0)
+    assert np.any(sf != sf6)
+    for f, slot in enumerate([4, 1, 2]):
+        np.testing.assert_array_equal(np_u8(cache.k_codes[slot]), codes[f])
+        np.testing.assert_array_equal(np_u8(cache.k_sf[slot]), sf[f])
+        np.testing.assert_array_equal(np_u8(cache.v_codes[slot]), codes[f])
+        assert float(cache.k_st[slot].item()) == float(st[f])
+    window = [2, 4, 1]
+    ko, _ = cache.dequant_window(window)
+    ref = orc.kv_dequant_window(np_u8(cache.k_codes), np_u8(cache.k_sf),
+                                cache.k_st.cpu().numpy(), window, tpf, heads, hd)
+    np.testing.assert_array_equal(bits(ko), ref)
+    assert nv.device_status() == 0
