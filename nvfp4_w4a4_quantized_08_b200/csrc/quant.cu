@@ -362,10 +362,31 @@ __device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, con
 }
 
 // ---- Four Over Six (KV chunks)
-// Magnitude of E2M1 code q (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6.
-__device__ __forceinline__ double e2m1_magnitude(uint32_t q) {
-  const double m = (q & 1) ? 1.5 : 1.0;
-  return q < 2 ? 0.5 * double(q) : ldexp(m, int(q >> 1) - 1);
+// Magnitude of E2M1 code q (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6, built from its
+// bits (code 1 = 0.5; codes 2..7 = (1 + (q & 1) / 2) * 2^(q / 2 - 1)).
+__device__ __forceinline__ float e2m1_magnitude(uint32_t q) {
+  const uint32_t bits = q < 2 ? (q ? 0x3F000000u : 0u)
+                              : ((126u + (q >> 1)) << 23) | ((q & 1u) << 22);
+  return __uint_as_float(bits);
+}
+
+// The same squared error in binary32 (v(q) * s_b exact, then one rounding per
+// operation).  Against the exact sum it is off by less than 2^-15.5 M^2 with
+// M = 2 amax_b (each |x| and each decoded value is below M): per element the
+// difference carries at most 2^-23 M, its square 2^-22 M^2 + 2^-24 M^2, and the
+// 16 additions 16 * 2^-24 * 16 M^2.
+__device__ __forceinline__ float block_sq_error_f32(const float a[16], uint2 codes, uint32_t sb,
+                                                    float s_t) {
+  const float sbv = e4m3_to_f32(sb & 0x7Fu);
+  float e = 0.0f;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    const uint32_t q = ((t < 8 ? codes.x : codes.y) >> (4 * (t & 7))) & 7u;
+    const float recon = __fmul_rn(__fmul_rn(e2m1_magnitude(q), sbv), s_t);
+    const float diff = __fsub_rn(fabsf(a[t]), recon);
+    e = __fadd_rn(e, __fmul_rn(diff, diff));
+  }
+  return e;
 }
 
 // Squared error of a block coded as (sb, codes) against the exactly decoded
@@ -382,7 +403,7 @@ __device__ __forceinline__ double block_sq_error(const RawBlock<InT>& raw, uint2
 #pragma unroll
   for (int t = 0; t < 16; ++t) {
     const uint32_t q = ((t < 8 ? codes.x : codes.y) >> (4 * (t & 7))) & 7u;
-    double recon = __dmul_rn(e2m1_magnitude(q), sbv);
+    double recon = __dmul_rn(double(e2m1_magnitude(q)), sbv);
     recon = __dmul_rn(recon, double(s_t));
     const double diff = __dsub_rn(double(fabsf(a[t])), recon);
     e = __dadd_rn(e, __dmul_rn(diff, diff));
@@ -390,8 +411,19 @@ __device__ __forceinline__ double block_sq_error(const RawBlock<InT>& raw, uint2
   return e;
 }
 
+// Out of line: the binary64 decision, for the rare blocks whose two binary32
+// errors are too close to order safely.
+template <typename InT>
+__device__ __noinline__ bool four_beats_six_exact(const RawBlock<InT> raw, uint2 c4, uint32_t sb4,
+                                                  uint2 c6, uint32_t sb6, float s_t) {
+  return block_sq_error<InT>(raw, c4, sb4, s_t) < block_sq_error<InT>(raw, c6, sb6, s_t);
+}
+
 // A block under Four Over Six: coded both ways (maximum onto 6 with k6, onto
-// 4 with k4), the one with the smaller squared error kept, 6 on a tie.
+// 4 with k4), the one with the smaller squared error kept, 6 on a tie.  The
+// errors are compared in binary32 when they differ by more than twice the
+// binary32 error bound (2^-12 amax_b^2 > 2 * 2^-15.5 (2 amax_b)^2), where the
+// order is certainly the binary64 one; otherwise in binary64.
 template <typename InT>
 __device__ __forceinline__ uint32_t quantize_block_4over6(const RawBlock<InT>& raw,
                                                           const float* inv_tab,
@@ -402,7 +434,18 @@ __device__ __forceinline__ uint32_t quantize_block_4over6(const RawBlock<InT>& r
   const uint32_t sb4 = quantize_block<InT>(raw, inv_tab, k4, c4);
   codes = c6;
   if (sb4 == sb6) return sb6;
-  if (block_sq_error<InT>(raw, c4, sb4, k6.s_t) < block_sq_error<InT>(raw, c6, sb6, k6.s_t)) {
+  float a[16];
+  unit_values<InT>(raw.h[0], a);
+  unit_values<InT>(raw.h[1], a + 8);
+  const float amax_b =
+      __uint_as_float(max(unit_absmax<InT>(raw.h[0]), unit_absmax<InT>(raw.h[1])));
+  const float e6 = block_sq_error_f32(a, c6, sb6, k6.s_t);
+  const float e4 = block_sq_error_f32(a, c4, sb4, k6.s_t);
+  const float margin = __fmul_rn(__fmul_rn(amax_b, amax_b), 0x1p-12f);
+  const bool four = fabsf(__fsub_rn(e4, e6)) > margin
+                        ? e4 < e6
+                        : four_beats_six_exact<InT>(raw, c4, sb4, c6, sb6, k6.s_t);
+  if (four) {
     codes = c4;
     return sb4;
   }
@@ -501,7 +544,7 @@ struct KvQuantArgs {
 };
 
 template <bool kContig, int kRule>
-__global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4 : 2)
+__global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4 : 3)
     kv_quant_kernel(KvQuantArgs args) {
   constexpr int D = Prefetch<__nv_bfloat16>::kDepth;
   __shared__ float inv_tab[128];

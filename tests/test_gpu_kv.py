@@ -149,3 +149,54 @@ def test_four_over_six_chunk_matches_oracle(orc, token_stride_extra):
                                 cache.k_st.cpu().numpy(), window, tpf, heads, hd)
     np.testing.assert_array_equal(bits(ko), ref)
     assert nv.device_status() == 0
+
+
+def _f32_steps_errors(blocks, s_t):
+    """Approximate (binary64) squared errors of each block under onto-6 and
+    onto-4, from the recipe's binary32 steps; used only to pick test blocks."""
+    import ml_dtypes
+    f32 = np.float32
+    amax_b = np.max(np.abs(blocks), axis=1).astype(f32)
+    out = []
+    for top in (6.0, 4.0):
+        r = amax_b / (f32(top) * f32(s_t))
+        sb = np.minimum(r, f32(448)).astype(ml_dtypes.float8_e4m3fn)
+        sbv = sb.astype(f32)
+        d = (sbv * f32(s_t))[:, None]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            y = np.clip(blocks / d, -6, 6)
+        q = y.astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+        q[sbv == 0] = 0
+        recon = np.abs(q) * sbv.astype(np.float64)[:, None] * float(s_t)
+        out.append((sb.view(np.uint8), ((np.abs(blocks) - recon) ** 2).sum(axis=1)))
+    return amax_b, out
+
+
+def test_four_over_six_near_ties_match_oracle(orc):
+    """Blocks whose two errors are within the binary32 screening margin (so
+    the kernel decides them in binary64), plus exact ties, plus ordinary
+    blocks: the chunk's scales and codes equal the oracle's."""
+    rng = np.random.default_rng(77)
+    s_t = np.float32(8.0) / np.float32(2688.0)
+    pool = rng.normal(0, 1, (40000, 16)) * rng.choice([0.3, 1.0, 2.5], (40000, 1))
+    pool = torch.from_numpy(np.clip(pool, -7.5, 7.5).astype(np.float32)).to(torch.bfloat16)
+    blocks = pool.float().numpy()
+    amax_b, ((s6, e6), (s4, e4)) = _f32_steps_errors(blocks, s_t)
+    near = np.nonzero((s4 != s6) & (np.abs(e4 - e6) <= 2.0 ** -12 * amax_b.astype(np.float64) ** 2))[0]
+    assert near.size >= 20
+    tie = np.zeros((2, 16), np.float32)
+    tie[0, :] = 3.0  # both rules code it exactly
+    tie[1, ::2] = 1.5
+    top = np.zeros((1, 16), np.float32)
+    top[0, 0] = 8.0  # the chunk's amax: s_t = 8 / 2688
+    chosen = np.concatenate([top, tie, blocks[near[:96]], blocks[:64]])
+    chunk = torch.from_numpy(chosen).to(torch.bfloat16)  # [tpf, heads=1, head_dim=16]
+    tpf = chunk.shape[0]
+    cache = nv.KVCache(2, tpf, 1, 16, scale_rule=nv.SCALE_FOUR_OVER_SIX)
+    d = chunk.reshape(tpf, 16).cuda()
+    cache.quant_chunk(d, d, [1])
+    codes, sf, st = orc.kv_quant_chunk(bits(chunk).reshape(-1), 1, tpf, 1, 16, rule=1)
+    assert float(st[0]) == float(s_t)
+    np.testing.assert_array_equal(np_u8(cache.k_sf[1]), sf[0])
+    np.testing.assert_array_equal(np_u8(cache.k_codes[1]), codes[0])
+    assert nv.device_status() == 0
