@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.orc_dequantize_exact.argtypes = [vp, vp, f32, i64, i64, vp]
         L.orc_gemm.restype = i32
         L.orc_gemm.argtypes = [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, i64, vp, vp]
+        L.orc_gelu_tanh.restype = i32
+        L.orc_gelu_tanh.argtypes = [vp, vp, i64]
         L.orc_kv_quant_chunk.restype = i32
         L.orc_kv_quant_chunk.argtypes = [vp, i64, i32, i32, i32, i32, vp, vp, vp, i32]
         L.orc_block_scale_rule.restype = i32
@@ -244,6 +246,15 @@ def gemm(a: Tuple[np.ndarray, np.ndarray, float], w: Tuple[np.ndarray, np.ndarra
                         K, None if ids is None else _ptr(ids), n, _ptr(y), _ptr(S))
     _check(rc, "gemm")
     return y, S
+
+
+def gelu_tanh(y: np.ndarray) -> np.ndarray:
+    """GELU, tanh form, elementwise in binary64 (the GEMM epilogue's FFN
+    activation): 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3)))."""
+    y = np.ascontiguousarray(y, np.float64)
+    out = np.empty_like(y)
+    _check(lib().orc_gelu_tanh(_ptr(y), _ptr(out), y.size), "gelu_tanh")
+    return out
 
 
 def kv_quant_chunk(kv: np.ndarray, n_frames: int, tpf: int, heads: int, head_dim: int,

@@ -39,6 +39,12 @@
  * (the standard rule) or onto 4, quantize with each, and keep the one whose
  * squared error against the exactly decoded values is smaller (ties keep 6).
  *
+ * FFN activation (GEMM epilogue option): GELU in its tanh form,
+ * 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))), in binary64 with the C
+ * library's tanh.  The DiT's blocks are attention and FFN (171host.com
+ * teardown, usage section "训练管线": LoRA on Attn/FFN); the pages name no
+ * activation, and the tanh form is the reading taken.
+ *
  * Parity pins (tests/test_oracle_*.py): exhaustive decode of all 16 E2M1 codes
  * and 256 E4M3 bytes against ml_dtypes / torch, encode against the same
  * libraries on tie and random values, exact round trips of representable
@@ -414,6 +420,21 @@ int orc_gemm(const uint8_t* a_codes, const uint8_t* a_sf, float a_st, const uint
     free(w);
   }
   free(a);
+  return ORC_OK;
+}
+
+
+/* GELU, tanh form, on n binary64 values: out[i] = 0.5 y (1 + tanh(c (y + 0.044715 y^3)))
+ * with c = sqrt(2 / pi), each operation one binary64 rounding. */
+int orc_gelu_tanh(const double* y, double* out, int64_t n) {
+  if (n < 0) return ORC_ERR_ARG;
+  const double c = sqrt(2.0 / 3.14159265358979323846);
+  for (int64_t i = 0; i < n; ++i) {
+    const double v = y[i];
+    if (!isfinite(v)) return ORC_ERR_NONFINITE;
+    const double inner = c * (v + 0.044715 * (v * v * v));
+    out[i] = 0.5 * v * (1.0 + tanh(inner));
+  }
   return ORC_OK;
 }
 

@@ -7,6 +7,30 @@ import torch
 
 GEMM_REL_TOL = 1e-3     # |y - y_ref| <= 1e-3 * sum_k |a_k w_k|
 BF16_HALF_ULP = 2.0 ** -8
+GELU_SLOPE_MAX = 1.13   # max |d GELU_tanh / dy| (pinned in test_oracle_gelu.py)
+TANH_APPROX_REL = 2.0 ** -11  # hardware tanh.approx.f32 relative error, with margin
+
+
+def assert_gelu_gemm_close(orc, g_gpu: np.ndarray, y_ref: np.ndarray, S: np.ndarray,
+                           bf16_out: bool):
+    """GEMM with the GELU epilogue: |g - GELU(y_ref)| <= GELU_SLOPE_MAX * e +
+    TANH_APPROX_REL * (|y_ref| + e) with e = 1e-3 * S (the GEMM bound carried
+    through GELU, plus the hardware tanh's error: the GELU differs by
+    0.5 |y| |dtanh|), plus half a bf16 ulp of the value for bf16 output."""
+    g_gpu = g_gpu.astype(np.float64)
+    g_ref = orc.gelu_tanh(y_ref)
+    e = GEMM_REL_TOL * S
+    tol = GELU_SLOPE_MAX * e + TANH_APPROX_REL * (np.abs(y_ref) + e)
+    if bf16_out:
+        tol = tol + BF16_HALF_ULP * (np.abs(g_ref) + tol)
+    err = np.abs(g_gpu - g_ref)
+    bad = ~(err <= tol)
+    if bad.any():
+        i = np.argwhere(bad)[:5]
+        raise AssertionError(
+            f"{bad.sum()} of {bad.size} outside tolerance; first {i.tolist()}: "
+            f"gpu {g_gpu[tuple(i[0])]} ref {g_ref[tuple(i[0])]} y_ref {y_ref[tuple(i[0])]} "
+            f"S {S[tuple(i[0])]}")
 
 
 def bits(x: torch.Tensor) -> np.ndarray:
