@@ -5,10 +5,11 @@ Step (per layer, on a 3-frame chunk of 2640 tokens; dim 3072, 24 heads x 128,
 FFN 14336): quantize the layer input -> QKV GEMM (N=9216) -> kv_quant_chunk of
 the 3 new frames' K and V straight out of the QKV output -> kv_dequant_window
 over 12 cached frames (3 sinks + 9 window) -> quantize the attention-output
-stand-in -> out-proj GEMM -> quantize -> FFN-up GEMM (N=14336) -> requantize
-the intermediate -> FFN-down GEMM; the down output feeds the next layer.
-Attention, norms, residuals and GELU are not part of the NVFP4 path and are not
-run; the attention output is a fixed seeded tensor.  Weights are pre-quantized
+stand-in -> out-proj GEMM -> quantize -> FFN-up GEMM (N=14336) with the GELU
+(tanh form) in its epilogue -> requantize the intermediate -> FFN-down GEMM;
+the down output feeds the next layer.  Attention, norms and residuals are not
+part of the NVFP4 path and are not run; the attention output is a fixed seeded
+tensor.  Weights are pre-quantized
 (outside the timed region).  The whole step is captured once as a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -154,7 +155,10 @@ class Step:
             mk("quant_act")
             nv.quantize(self.o_out, out=self.qa, ws=self.ws, amax_in=a_o)
             mk("gemm_up")
-            nv.gemm(self.qa, wu, out=self.up_out, ws=self.ws, c_amax=a_u)
+            # FFN up-projection with its GELU in the epilogue; the stored GELU
+            # output's amax feeds the intermediate requantization
+            nv.gemm(self.qa, wu, out=self.up_out, ws=self.ws, c_amax=a_u,
+                    act=nv.ACT_GELU_TANH)
             mk("requant_ffn")
             nv.quantize(self.up_out, out=self.qf, ws=self.ws, amax_in=a_u)
             mk("gemm_down")
@@ -341,8 +345,9 @@ def config_block(args):
             "global_batch": M * max(1, args.gpus), "seq_len": M,
             "parallelism": f"replica{args.gpus}" if args.gpus > 1 else "single",
             "l2": "inputs larger than L2 (2.1 GB NVFP4 weights + 1.4 GB KV pools per step)",
-            "stand_ins": "attention output fixed seeded tensor; attention, norm, residual, "
-                         "GELU not run (outside the NVFP4 path)"}
+            "stand_ins": "attention output fixed seeded tensor; attention, norm, residual "
+                         "not run (outside the NVFP4 path); FFN GELU (tanh form) fused in the "
+                         "up-projection epilogue"}
 
 
 def time_kv_four_over_six(step: "Step", dev, reps: int = 20) -> float:

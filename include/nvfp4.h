@@ -90,6 +90,21 @@ typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA128x4 = 1 } nvfp4_sf_layout;
  *     element order; 6 on a tie).  The stored format is unchanged. */
 typedef enum { NVFP4_SCALE_ONTO_6 = 0, NVFP4_SCALE_FOUR_OVER_SIX = 1 } nvfp4_scale_rule;
 
+/* Elementwise function the GEMM epilogue applies to y = (s_tA * s_tW) * acc
+ * before rounding to the output type.
+ *   NONE: C = y.
+ *   GELU_TANH: C = 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))), the GELU of
+ *     the DiT's FFN between its up- and down-projection (the transformer blocks
+ *     are attention and FFN: 171host.com LongLive-2.0 teardown, usage section
+ *     "训练管线", LoRA on Attn/FFN); the pages name no activation form, the
+ *     tanh form is the one video DiTs use.  Evaluated in binary32 with the
+ *     hardware tanh (tanh.approx.f32, relative error about 2^-11) on y as a
+ *     bf16 linear layer hands it to its activation: for bf16 output on y
+ *     rounded to bf16, for fp32 output on the fp32 y.  So C is within
+ *     2^-11 |y| + 1.13 |y_in - y_exact| of the exact GELU of the exact y, with
+ *     y_in the activation's input, plus the output rounding. */
+typedef enum { NVFP4_ACT_NONE = 0, NVFP4_ACT_GELU_TANH = 1 } nvfp4_act;
+
 /* An NVFP4 tensor of rows x cols elements (cols a multiple of 16).
  *   codes: device, [rows][cols/2] bytes; element 2j in the low nibble of
  *          byte j, element 2j+1 in the high nibble; sign in bit 3 of a nibble.
@@ -178,16 +193,18 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64
 /* Block-scaled FP4 x FP4 GEMM, C = A * W^T:
  *   C[m][n] = (s_tA * s_tW) * sum_k v(qA[m][k]) sA[m][k/16] * v(qW[n][k]) sW[n][k/16]
  * products and sums on the tensor cores with FP32 accumulation, the scale
- * product applied once in the epilogue, then rounded to c_dtype.
+ * product applied once in the epilogue, then the activation `act`
+ * (nvfp4_act), then rounded to c_dtype.
  *   A: M x K activations, W: N x K weights (both K-contiguous), both with
  *      sf_layout == NVFP4_SF_MMA128x4 and the same K.
  *   Shapes: K a multiple of 64, N a multiple of 256, M >= 1 (any M; tail rows
  *      are masked).
  *   C: device, c_dtype (bf16 or fp32), row stride ldc >= N elements, ldc a
  *      multiple of 8, 16-byte aligned.
+ *   act: nvfp4_act.
  *   c_amax: NULL, or device floats (4-byte aligned) into which the GEMM
- *      max-accumulates max|C| over the values as stored (after rounding to
- *      c_dtype), so that nvfp4_quantize(..., amax_in = c_amax, ...) can
+ *      max-accumulates max|C| over the values as stored (after the activation
+ *      and the rounding to c_dtype), so that nvfp4_quantize(..., amax_in = c_amax, ...) can
  *      requantize C without an amax pass.  With c_amax_cols == 0 there is one
  *      word for all of C; with c_amax_cols > 0 (a multiple of 256 dividing N)
  *      word g covers columns [g * c_amax_cols, (g + 1) * c_amax_cols), N /
@@ -200,7 +217,7 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, ARCH, CUDA;
  * TIMEOUT via the status word. */
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C,
-                                  int32_t c_dtype, int64_t ldc, float* c_amax,
+                                  int32_t c_dtype, int64_t ldc, int32_t act, float* c_amax,
                                   int64_t c_amax_cols, void* ws, size_t ws_bytes, void* stream);
 
 /* Quantize one chunk of n_frames (1..8) new latent frames of K and V into the

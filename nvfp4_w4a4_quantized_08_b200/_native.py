@@ -29,6 +29,8 @@ SF_ROWMAJOR = 0
 SF_MMA128x4 = 1
 SCALE_ONTO_6 = 0
 SCALE_FOUR_OVER_SIX = 1
+ACT_NONE = 0
+ACT_GELU_TANH = 1
 KV_MAX_CHUNK_FRAMES = 8
 KV_MAX_WINDOW_SLOTS = 256
 
@@ -87,7 +89,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_dequantize.restype = i32
         L.nvfp4_dequantize.argtypes = [TP, vp, i64, vp]
         L.nvfp4_gemm.restype = i32
-        L.nvfp4_gemm.argtypes = [TP, TP, vp, i32, i64, vp, i64, vp, sz, vp]
+        L.nvfp4_gemm.argtypes = [TP, TP, vp, i32, i64, i32, vp, i64, vp, sz, vp]
         L.nvfp4_kv_quant_chunk.restype = i32
         L.nvfp4_kv_quant_chunk.argtypes = [KP, vp, vp, i64, ctypes.POINTER(ctypes.c_int32), i32,
                                              vp, vp, vp, sz, vp]

@@ -157,13 +157,14 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64_t ld, voi
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, int32_t c_dtype,
-                        int64_t ldc, float* c_amax, int64_t c_amax_cols, void* ws,
+                        int64_t ldc, int32_t act, float* c_amax, int64_t c_amax_cols, void* ws,
                         size_t ws_bytes, void* stream) {
   nvfp4_status st = check_tensor(A);
   if (st != NVFP4_OK) return st;
   st = check_tensor(W);
   if (st != NVFP4_OK) return st;
   if (!C || (c_dtype != NVFP4_BF16 && c_dtype != NVFP4_FP32)) return NVFP4_ERR_INVALID_ARG;
+  if (act != NVFP4_ACT_NONE && act != NVFP4_ACT_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
   if (A->sf_layout != NVFP4_SF_MMA128x4 || W->sf_layout != NVFP4_SF_MMA128x4)
     return NVFP4_ERR_INVALID_ARG;
   if (A->cols != W->cols) return NVFP4_ERR_INVALID_ARG;
@@ -192,6 +193,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
   g.c = C;
   g.c_dtype = c_dtype;
   g.ldc = ldc;
+  g.act = act;
   g.c_amax = c_amax;
   g.c_amax_cols = c_amax_cols;
   g.ws = ws;

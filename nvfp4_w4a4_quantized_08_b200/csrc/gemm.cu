@@ -223,10 +223,33 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   return v;
 }
 
+// GELU, tanh form: 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), in
+// binary32 with the hardware tanh (relative error about 2^-11).
+__device__ __forceinline__ float gelu_tanh(float v) {
+  const float u = __fmul_rn(v, __fmaf_rn(0.0356774081f, __fmul_rn(v, v), 0.7978845608f));
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(u));
+  const float h = __fmul_rn(0.5f, v);
+  return __fmaf_rn(h, t, h);
+}
+
+// The epilogue's function of y = alpha * acc (fp32 output).
+template <bool kGelu>
+__device__ __forceinline__ float epi(float acc, float alpha) {
+  const float y = __fmul_rn(acc, alpha);
+  return kGelu ? gelu_tanh(y) : y;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// GELU of both bf16 halves of a word, rounded back to bf16.
+__device__ __forceinline__ uint32_t gelu_bf16x2(uint32_t w) {
+  return bf16x2_rn(gelu_tanh(__uint_as_float(w << 16)),
+                   gelu_tanh(__uint_as_float(w & 0xFFFF0000u)));
 }
 
 // ---------------------------------------------------------------- bounded waits
@@ -327,6 +350,7 @@ struct Params {
   int32_t c_dtype;
 };
 
+template <bool kGelu>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                       const __grid_constant__ CUtensorMap map_w,
@@ -502,8 +526,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     // The accumulator is read out whole into registers (bf16: 128 packed words
-    // a thread; fp32: two halves of 128 words) and released to the MMA issuer
-    // before the stores, so the next tile's MMAs wait only for the reads.
+    // a thread; fp32: two halves of 128 words), scaled by s_tA * s_tW and
+    // released to the MMA issuer before the stores, so the next tile's MMAs
+    // wait only for the reads.  The activation (kGelu) takes the bf16 products
+    // after the release (fp32 output: the fp32 products, as they are read).
     const uint32_t ew = uint32_t(warp - 2);            // staging buffers of this warp
     const uint32_t quad = uint32_t(warp & 3);          // tensor-memory lane quadrant
     const float alpha = __fmul_rn(*p.a_st, *p.w_st);
@@ -549,6 +575,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) bar_arrive(bar_acc_release);
+        // the activation runs on the bf16 products once the accumulator is
+        // released, overlapping the next tile's MMAs: a bf16 linear layer
+        // followed by its activation
+        if (kGelu) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) pk[e] = gelu_bf16x2(pk[e]);
+        }
         if (row_live) {
 #pragma unroll
           for (int e = 0; e < 128; ++e) vmax = __vmaxu2(vmax, pk[e] & 0x7FFF7FFFu);
@@ -567,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(taddr + 128 * half + 32 * c, r);
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              v[32 * c + e] = __float_as_uint(__fmul_rn(__uint_as_float(r[e]), alpha));
+              v[32 * c + e] = __float_as_uint(epi<kGelu>(__uint_as_float(r[e]), alpha));
           }
           if (half == 1) {
             tc_fence_before();
@@ -653,17 +686,25 @@ static bool make_out_map(CUtensorMap* map, void* base, int32_t dtype, uint64_t r
   return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
+template <bool kGelu>
+static cudaError_t launch_form(const CUtensorMap& map_a, const CUtensorMap& map_w,
+                               const CUtensorMap& map_c, const gemm::Params& p, int grid,
+                               cudaStream_t st) {
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel,
+    cudaError_t e = cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel<kGelu>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          gemm::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
+  return launch_pdl(gemm::nvfp4_gemm_kernel<kGelu>, dim3(grid), dim3(gemm::kThreads),
+                    size_t(gemm::kSmemBytes), st, map_a, map_w, map_c, p);
+}
+
+cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   CUtensorMap map_a, map_w, map_c;
   if (!make_code_map(&map_a, g.a_codes, uint64_t(g.K / 2), uint64_t(g.M), gemm::kBM) ||
       !make_code_map(&map_w, g.w_codes, uint64_t(g.K / 2), uint64_t(g.N), gemm::kBN) ||
@@ -687,8 +728,8 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.c_dtype = g.c_dtype;
   const uint32_t tiles = p.tiles_m * p.tiles_n;
   const int grid = int(tiles < uint32_t(g.sm_count) ? tiles : uint32_t(g.sm_count));
-  return launch_pdl(gemm::nvfp4_gemm_kernel, dim3(grid), dim3(gemm::kThreads),
-                    size_t(gemm::kSmemBytes), st, map_a, map_w, map_c, p);
+  return g.act == NVFP4_ACT_GELU_TANH ? launch_form<true>(map_a, map_w, map_c, p, grid, st)
+                                      : launch_form<false>(map_a, map_w, map_c, p, grid, st);
 }
 
 }  // namespace nvfp4

@@ -72,6 +72,7 @@ struct LaunchGemm {
   void* c;
   int32_t c_dtype;
   int64_t ldc;
+  int32_t act;    // nvfp4_act applied in the epilogue
   float* c_amax;  // max|C| accumulator(s), or NULL
   int64_t c_amax_cols;  // columns per accumulator word (0: one word)
   void* ws;

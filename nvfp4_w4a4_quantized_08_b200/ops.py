@@ -121,8 +121,12 @@ def dequantize(t: NVFP4Tensor, out: Optional[torch.Tensor] = None) -> torch.Tens
 
 def gemm(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype: torch.dtype = torch.bfloat16,
          out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-         c_amax: Optional[torch.Tensor] = None, c_amax_cols: int = 0) -> torch.Tensor:
-    """nvfp4_gemm: C = A W^T, [a.rows, w.rows] in bf16 or fp32.
+         c_amax: Optional[torch.Tensor] = None, c_amax_cols: int = 0,
+         act: int = N.ACT_NONE) -> torch.Tensor:
+    """nvfp4_gemm: C = act(A W^T), [a.rows, w.rows] in bf16 or fp32.
+
+    act:    N.ACT_NONE, or N.ACT_GELU_TANH (the FFN's GELU, tanh form, in the
+            epilogue before the output rounding).
 
     c_amax: fp32 tensor that starts at 0 (or at a smaller running max); the
             kernel raises it to max|C| over the values it stores.  With
@@ -139,7 +143,7 @@ def gemm(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype: torch.dtype = torch.bfloat16
     ws = workspace(a.device) if ws is None else ws
     sa, sw = a.c_struct(), w.c_struct()
     N.check(N.lib().nvfp4_gemm(ctypes.byref(sa), ctypes.byref(sw), out.data_ptr(),
-                               _dtype_code(out), out.stride(0), _ptr(c_amax), c_amax_cols,
+                               _dtype_code(out), out.stride(0), act, _ptr(c_amax), c_amax_cols,
                                ws.data_ptr(), ws.numel(), _stream()), "nvfp4_gemm")
     return out
 

@@ -14,12 +14,16 @@ TANH_APPROX_REL = 2.0 ** -11  # hardware tanh.approx.f32 relative error, with ma
 def assert_gelu_gemm_close(orc, g_gpu: np.ndarray, y_ref: np.ndarray, S: np.ndarray,
                            bf16_out: bool):
     """GEMM with the GELU epilogue: |g - GELU(y_ref)| <= GELU_SLOPE_MAX * e +
-    TANH_APPROX_REL * (|y_ref| + e) with e = 1e-3 * S (the GEMM bound carried
-    through GELU, plus the hardware tanh's error: the GELU differs by
-    0.5 |y| |dtanh|), plus half a bf16 ulp of the value for bf16 output."""
+    TANH_APPROX_REL * (|y_ref| + e), e the error of GELU's input: the GEMM
+    bound 1e-3 * S, plus for bf16 output the rounding of y to bf16 (the GELU
+    takes the bf16 product there), carried through GELU's slope; the second
+    term is the hardware tanh's error (the GELU moves by 0.5 |y| |dtanh|).
+    For bf16 output, half a bf16 ulp of the result on top."""
     g_gpu = g_gpu.astype(np.float64)
     g_ref = orc.gelu_tanh(y_ref)
     e = GEMM_REL_TOL * S
+    if bf16_out:
+        e = e + BF16_HALF_ULP * (np.abs(y_ref) + e)
     tol = GELU_SLOPE_MAX * e + TANH_APPROX_REL * (np.abs(y_ref) + e)
     if bf16_out:
         tol = tol + BF16_HALF_ULP * (np.abs(g_ref) + tol)

@@ -89,7 +89,7 @@ def test_gemm_rejects(L):
     a = _tensor(rows=2640, cols=3072)
     w = _tensor(rows=9216, cols=3072)
     g = L.nvfp4_gemm
-    ok_args = (FAKE, N.BF16, 9216, None, 0, FAKE, 256, None)
+    ok_args = (FAKE, N.BF16, 9216, N.ACT_NONE, None, 0, FAKE, 256, None)
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9216, cols=3072, layout=N.SF_ROWMAJOR)),
              *ok_args) == N.ERR_INVALID_ARG
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9216, cols=2048)),
@@ -97,19 +97,22 @@ def test_gemm_rejects(L):
     assert g(ctypes.byref(_tensor(rows=2640, cols=3056)),
              ctypes.byref(_tensor(rows=9216, cols=3056)), *ok_args) == N.ERR_UNSUPPORTED_SHAPE
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9200, cols=3072)),
-             FAKE, N.BF16, 9216, None, 0, FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # N % 256
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9000, None, 0, FAKE, 256,
+             FAKE, N.BF16, 9216, 0, None, 0, FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # N % 256
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9000, 0, None, 0, FAKE, 256,
              None) == N.ERR_INVALID_ARG  # ldc < N
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9220, None, 0, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9220, 0, None, 0, FAKE, 256,
              None) == N.ERR_MISALIGNED
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, 5, 9216, None, 0, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, 5, 9216, 0, None, 0, FAKE, 256,
              None) == N.ERR_INVALID_ARG
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, None, 0, FAKE, 4,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, 0, None, 0, FAKE, 4,
              None) == N.ERR_WORKSPACE
-    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, FAKE + 1, 0, FAKE, 256,
+    assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, 0, FAKE + 1, 0, FAKE, 256,
              None) == N.ERR_MISALIGNED  # c_amax
     for cols in (-256, 100, 2048, 9216 * 2):  # not a multiple of 256 dividing N
-        assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, FAKE, cols, FAKE, 256,
+        assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, 0, FAKE, cols, FAKE, 256,
+                 None) == N.ERR_INVALID_ARG
+    for act in (-1, 2):  # not an nvfp4_act
+        assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9216, act, None, 0, FAKE, 256,
                  None) == N.ERR_INVALID_ARG
 
 

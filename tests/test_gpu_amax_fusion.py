@@ -92,6 +92,23 @@ def test_gemm_to_quantize_chain(orc):
     assert torch.equal(q2.codes, ref.codes) and torch.equal(q2.s_t, ref.s_t)
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gelu_epilogue_amax_and_requant(orc, out_dtype):
+    """FFN up-projection with the GELU epilogue feeding the intermediate
+    requantization: c_amax is exactly max|C| of the stored GELU values, and the
+    quantization fed from it is the one the oracle makes of those values."""
+    qa, qw = _operands(390, 1024, 512, seed=51)
+    word = _amax_word()
+    h = nv.gemm(qa, qw, out_dtype=out_dtype, c_amax=word, act=nv.ACT_GELU_TANH)
+    torch.cuda.synchronize()
+    assert word.item() == h.float().abs().max().item()
+    assert h.float().min().item() > -0.171  # GELU's floor
+    q = nv.quantize(h, amax_in=word)
+    assert word.item() == 0.0
+    assert_quant_equal(orc, q, bits(h), nv.SF_MMA128x4)
+    assert nv.device_status() == 0
+
+
 def test_amax_in_out_of_domain_is_reported_and_reset():
     x = torch.ones(64, 64, device="cuda", dtype=torch.bfloat16)
     word = torch.full((1,), 1e38, dtype=torch.float32, device="cuda")  # s_t > 2^100

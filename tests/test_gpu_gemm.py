@@ -11,7 +11,7 @@ import torch
 import nvfp4_w4a4_quantized_08_b200 as nv
 from nvfp4_w4a4_quantized_08_b200 import workloads as wl
 
-from _util import assert_gemm_close, assert_quant_equal, bits
+from _util import assert_gelu_gemm_close, assert_gemm_close, assert_quant_equal, bits
 
 pytestmark = pytest.mark.gpu
 
@@ -105,6 +105,35 @@ def test_ffn_pair(orc):
     rows = _sample_rows(f.h.shape[0], n_random=16, seed=2)
     y_ref, S = orc.gemm(oh, od, rows=rows)
     assert_gemm_close(y_dn[rows].float().cpu().numpy(), y_ref, S, True)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (129, 512, 320), (300, 768, 1024)])
+def test_gelu_epilogue(orc, M, N, K, out_dtype):
+    """act = GELU (tanh form) in the epilogue, every element against the
+    oracle's binary64 GELU of its binary64 GEMM, over inputs that put outputs
+    on both sides of zero and far out in the tails."""
+    g = torch.Generator().manual_seed(M + 3 * N + 5 * K)
+    a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.1).to(torch.bfloat16)
+    qa, qw, oa, ow = _operands(orc, a, w)
+    y = nv.gemm(qa, qw, out_dtype=out_dtype, act=nv.ACT_GELU_TANH)
+    y_ref, S = orc.gemm(oa, ow)
+    assert (y_ref < -3).any() and (y_ref > 3).any()
+    assert_gelu_gemm_close(orc, y.float().cpu().numpy(), y_ref, S, out_dtype == torch.bfloat16)
+    assert nv.device_status() == 0
+
+
+def test_ffn_up_with_gelu(orc):
+    """FFN up-projection M=2640, N=14336, K=3072 with the GELU epilogue, bf16
+    output, sampled rows (all columns, the ragged last tile included)."""
+    f = wl.ffn()
+    qx, qu, ox, ou = _operands(orc, f.x, f.w_up)
+    h = nv.gemm(qx, qu, out_dtype=torch.bfloat16, act=nv.ACT_GELU_TANH)
+    rows = _sample_rows(f.x.shape[0], n_random=12, seed=3)
+    y_ref, S = orc.gemm(ox, ou, rows=rows)
+    assert_gelu_gemm_close(orc, h[rows].float().cpu().numpy(), y_ref, S, True)
+    assert nv.device_status() == 0
 
 
 def test_timeout_path_reports_and_recovers(orc):
