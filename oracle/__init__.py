@@ -85,6 +85,9 @@ def lib() -> ctypes.CDLL:
         L.orc_dequantize_exact.argtypes = [vp, vp, f32, i64, i64, vp]
         L.orc_gemm.restype = i32
         L.orc_gemm.argtypes = [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, i64, vp, vp]
+        L.orc_window_attention.restype = i32
+        L.orc_window_attention.argtypes = [vp, i64, vp, i64, vp, vp, i64, i32, i32,
+                                           ctypes.c_double, vp, vp]
         L.orc_gelu_tanh.restype = i32
         L.orc_gelu_tanh.argtypes = [vp, vp, i64]
         L.orc_kv_quant_chunk.restype = i32
@@ -299,3 +302,27 @@ def kv_dequant_window(pool_codes: np.ndarray, pool_sf: np.ndarray, pool_st: np.n
                                      head_dim, _ptr(out))
     _check(rc, "kv_dequant_window")
     return out
+
+
+def window_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                     rows: Optional[Sequence[int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Windowed attention in binary64.  q: bf16 bits [tq, q_stride] (head h at
+    columns h*head_dim...); k, v: bf16 bits [n_kv, heads, head_dim] (the window
+    rebuild's output).  -> (out, E), both [n_rows, heads, head_dim]:
+    out = sum_j p_j v_j, E = sum_j p_j |v_j| (the scale of the P V sum)."""
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    n_kv, heads, hd = k.shape
+    assert v.shape == k.shape and q.ndim == 2
+    if rows is None:
+        ids, n = None, q.shape[0]
+    else:
+        ids = np.ascontiguousarray(np.asarray(rows, np.int64))
+        n = ids.shape[0]
+    out = np.empty((n, heads, hd), np.float64)
+    E = np.empty((n, heads, hd), np.float64)
+    _check(lib().orc_window_attention(_ptr(q), q.shape[1], None if ids is None else _ptr(ids), n,
+                                      _ptr(k), _ptr(v), n_kv, heads, hd, float(scale), _ptr(out),
+                                      _ptr(E)), "window_attention")
+    return out, E

@@ -45,6 +45,12 @@
  * teardown, usage section "训练管线": LoRA on Attn/FFN); the pages name no
  * activation, and the tanh form is the reading taken.
  *
+ * Windowed attention over the cache (the consumer of the window rebuild:
+ * hyper.ai summary, section "方法"; 3 sinks + 9 window frames, 171host.com
+ * section 2.2): out = softmax(scale * q k^T) v over the window's tokens in
+ * slot-list order, every query seeing every window token, in binary64 on the
+ * bf16 K and V the window rebuild produces.
+ *
  * Parity pins (tests/test_oracle_*.py): exhaustive decode of all 16 E2M1 codes
  * and 256 E4M3 bytes against ml_dtypes / torch, encode against the same
  * libraries on tie and random values, exact round trips of representable
@@ -488,4 +494,59 @@ int orc_kv_dequant_window(const uint8_t* pool_codes, const uint8_t* pool_sf, con
     if (rc) return rc;
   }
   return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* windowed attention                                                  */
+/* ------------------------------------------------------------------ */
+
+static double bf16_value(uint16_t b) { return (double)f32_from_bits((uint32_t)b << 16); }
+
+/* q: bf16 bits, token t at q + t*q_stride, head h at +h*head_dim; k, v: bf16
+ * bits [n_kv][heads][head_dim].  For each requested query token rows[r] (all
+ * 0..n_rows-1 when rows is NULL) and head h:
+ *   p_j = exp(scale * sum_d q[d] k_j[d] - max_j(...)) / sum_j exp(...),
+ *   out[r][h][d] = sum_j p_j v_j[d],   E[r][h][d] = sum_j p_j |v_j[d]|,
+ * each sum in index order, binary64. */
+int orc_window_attention(const uint16_t* q, int64_t q_stride, const int64_t* rows, int64_t n_rows,
+                         const uint16_t* k, const uint16_t* v, int64_t n_kv, int heads,
+                         int head_dim, double scale, double* out, double* E) {
+  if (n_rows < 0 || n_kv < 1 || heads < 1 || head_dim < 1 || !(scale > 0.0)) return ORC_ERR_ARG;
+  int err = ORC_OK;
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    const int64_t t = rows ? rows[r] : r;
+    double* logit = (double*)malloc((size_t)n_kv * sizeof(double));
+    if (!logit) { err = ORC_ERR_ARG; continue; }
+    for (int h = 0; h < heads; ++h) {
+      const uint16_t* qh = q + t * q_stride + (int64_t)h * head_dim;
+      double mx = -INFINITY;
+      for (int64_t j = 0; j < n_kv; ++j) {
+        const uint16_t* kj = k + (j * heads + h) * (int64_t)head_dim;
+        double dot = 0.0;
+        for (int d = 0; d < head_dim; ++d) dot += bf16_value(qh[d]) * bf16_value(kj[d]);
+        logit[j] = scale * dot;
+        if (logit[j] > mx) mx = logit[j];
+      }
+      double sum = 0.0;
+      for (int64_t j = 0; j < n_kv; ++j) {
+        logit[j] = exp(logit[j] - mx);
+        sum += logit[j];
+      }
+      double* o = out + (r * heads + h) * (int64_t)head_dim;
+      double* e = E + (r * heads + h) * (int64_t)head_dim;
+      for (int d = 0; d < head_dim; ++d) o[d] = e[d] = 0.0;
+      for (int64_t j = 0; j < n_kv; ++j) {
+        const double p = logit[j] / sum;
+        const uint16_t* vj = v + (j * heads + h) * (int64_t)head_dim;
+        for (int d = 0; d < head_dim; ++d) {
+          const double x = bf16_value(vj[d]);
+          o[d] += p * x;
+          e[d] += p * fabs(x);
+        }
+      }
+    }
+    free(logit);
+  }
+  return err;
 }
