@@ -350,6 +350,38 @@ def config_block(args):
                          "up-projection epilogue"}
 
 
+ATTN_FLOPS = 4 * M * WINDOW * TPF * wl.HEAD_DIM * wl.HEADS  # QK^T and PV, one layer
+
+
+def time_window_attention(step: "Step", dev, reps: int = 10) -> float:
+    """Device ms of one nvfp4_window_attention: the chunk's 2640 queries (the Q
+    third of the QKV output) over layer 0's 12-slot window read from the NVFP4
+    pools, graph-replayed."""
+    cache = step.cache[0]
+    q = step.qkv_out[:, :D]
+    out = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            cache.window_attention(q, step.window, out=out)
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):
+                cache.window_attention(q, step.window, out=out)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    del g
+    return e0.elapsed_time(e1) / reps
+
+
 def time_kv_four_over_six(step: "Step", dev, reps: int = 20) -> float:
     """Device ms of one nvfp4_kv_quant_chunk (3 frames of K and V read from a
     QKV output, amax pass included) with the Four Over Six scale rule."""
@@ -482,6 +514,9 @@ def run_ours(args):
     # the KV chunk under Four Over Six (the adaptive KV scale rule; not on the
     # step's path): one layer's 3 new frames of K and V, graph-replayed
     fos_ms = time_kv_four_over_six(step, dev)
+    # attention over the window straight from the NVFP4 pools (the window
+    # rebuild's consumer; the step itself keeps a fixed attention output)
+    attn_ms = time_window_attention(step, dev)
 
     peaks, peak_src = measured_peaks()
     fp4_peak = 4.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -523,6 +558,11 @@ def run_ours(args):
                 "gb_s": CODEC_BYTES["kv_quant"] / (fos_ms * 1e-3) / 1e9,
                 "frac_hbm": CODEC_BYTES["kv_quant"] / (fos_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "vs_onto_6_us": kernel_ms["kv_quant"] / args.layers * 1e3},
+            "window_attention": {
+                "us": attn_ms * 1e3, "tflops": ATTN_FLOPS / (attn_ms * 1e-3) / 1e12,
+                "bound": "tensor (bf16 mma.sync)",
+                "frac_bf16_peak": ATTN_FLOPS / (attn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "shape": f"{M} queries x {WINDOW * TPF} keys x {wl.HEADS} heads x {wl.HEAD_DIM}"},
             "gemm": {"tflops": gemm_tflops, "ms_per_step": gemm_ms,
                      "launches_per_step": gemm_launches,
                      "by_shape_ms": {k: v for k, v in kernel_ms.items() if k.startswith("gemm")}},

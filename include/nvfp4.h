@@ -253,6 +253,29 @@ NVFP4_API nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const v
 NVFP4_API nvfp4_status nvfp4_kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slot_ids,
                                      int32_t n, void* k_out, void* v_out, void* stream);
 
+/* Windowed attention straight from the NVFP4 cache (the consumer of the window
+ * rebuild above, without the bf16 round trip through HBM):
+ *   out[t][h] = sum_j softmax_j(softmax_scale * q[t][h] . k[j][h]) v[j][h]
+ * over the tokens j of the listed slots in list order, k and v the bf16 values
+ * nvfp4_kv_dequant_window would write (bf16_RNE((v(q) * s_b) * s_t)); every
+ * query sees every window token (the chunk attends to the cached frames and to
+ * itself whole).  Scores and sums in fp32 (tensor cores, bf16 inputs), the
+ * probabilities rounded to bf16 for the P V product, the output rounded to bf16.
+ *   slot_ids: host, n ids in [0, n_slots), 1 <= n <= NVFP4_KV_MAX_WINDOW_SLOTS,
+ *             n * tokens_per_frame < 2^31; repeats allowed.
+ *   q:   device bf16, tq tokens (1 <= tq <= 2^30), token t at q + t *
+ *        q_token_stride elements, heads x head_dim contiguous in a token
+ *        (q_token_stride >= heads * head_dim, a multiple of 8), 16-byte aligned;
+ *        this reads Q straight out of a fused QKV projection output.
+ *   softmax_scale: finite, > 0 (usually 1 / sqrt(head_dim)).
+ *   out: device bf16, tq tokens at out_token_stride, same layout as q.
+ *   head_dim must be 128.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, ARCH, CUDA. */
+NVFP4_API nvfp4_status nvfp4_window_attention(const nvfp4_kv_cache* cache, const int32_t* slot_ids,
+                                              int32_t n, const void* q, int64_t q_token_stride,
+                                              int64_t tq, float softmax_scale, void* out,
+                                              int64_t out_token_stride, void* stream);
+
 /* Size of the library-owned scratch array behind nvfp4_quantize_noalloc. */
 #define NVFP4_NOALLOC_SCRATCH_BYTES 256
 

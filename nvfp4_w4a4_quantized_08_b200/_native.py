@@ -38,7 +38,7 @@ EXPORTS = (
     "nvfp4_codes_bytes", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
     "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_quant_chunk", "nvfp4_kv_dequant_window",
     "nvfp4_get_device_status", "nvfp4_set_wait_limit_ns", "nvfp4_status_string",
-    "nvfp4_quantize_noalloc",
+    "nvfp4_quantize_noalloc", "nvfp4_window_attention",
 )
 
 
@@ -95,6 +95,9 @@ def lib() -> ctypes.CDLL:
                                              vp, vp, vp, sz, vp]
         L.nvfp4_kv_dequant_window.restype = i32
         L.nvfp4_kv_dequant_window.argtypes = [KP, ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
+        L.nvfp4_window_attention.restype = i32
+        L.nvfp4_window_attention.argtypes = [KP, ctypes.POINTER(ctypes.c_int32), i32, vp, i64,
+                                             i64, ctypes.c_float, vp, i64, vp]
         L.nvfp4_get_device_status.restype = i32
         L.nvfp4_get_device_status.argtypes = [vp, vp]
         L.nvfp4_set_wait_limit_ns.restype = None

@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libnvfp4 (declared in include/nvfp4.h): host-side
 // argument checks, then one or two kernel launches on the caller's stream.
+#include <cmath>
 #include <atomic>
 #include <cstring>
 
@@ -277,6 +278,47 @@ nvfp4_status nvfp4_kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t*
   d.v_out = v_out;
   d.sm_count = dev.sm_count;
   return cuda_status(launch_kv_dequant(d, static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_window_attention(const nvfp4_kv_cache* cache, const int32_t* slot_ids,
+                                    int32_t n, const void* q, int64_t q_token_stride, int64_t tq,
+                                    float softmax_scale, void* out, int64_t out_token_stride,
+                                    void* stream) {
+  nvfp4_status st = check_cache(cache);
+  if (st != NVFP4_OK) return st;
+  if (!slot_ids || !q || !out || n < 1 || n > NVFP4_KV_MAX_WINDOW_SLOTS)
+    return NVFP4_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (slot_ids[i] < 0 || slot_ids[i] >= cache->n_slots) return NVFP4_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return NVFP4_ERR_INVALID_ARG;
+  const int64_t row = int64_t(cache->heads) * cache->head_dim;
+  if (q_token_stride < row || out_token_stride < row) return NVFP4_ERR_INVALID_ARG;
+  if (cache->head_dim != 128 || tq < 1 || tq > (int64_t(1) << 30) || cache->heads > 65535 ||
+      int64_t(n) * cache->tokens_per_frame >= (int64_t(1) << 31))
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(q, 16) || !aligned(out, 16) || q_token_stride % 8 != 0 ||
+      out_token_stride % 8 != 0)
+    return NVFP4_ERR_MISALIGNED;
+  const DeviceInfo dev = current_device();
+  if (!dev.ok) return NVFP4_ERR_ARCH;
+  LaunchAttn d;
+  d.k_codes = cache->k_codes;
+  d.v_codes = cache->v_codes;
+  d.k_sf = cache->k_sf;
+  d.v_sf = cache->v_sf;
+  d.k_st = cache->k_st;
+  d.v_st = cache->v_st;
+  d.slot_ids = slot_ids;
+  d.n = n;
+  d.tpf = cache->tokens_per_frame;
+  d.heads = cache->heads;
+  d.q = q;
+  d.out = out;
+  d.q_stride = q_token_stride;
+  d.out_stride = out_token_stride;
+  d.tq = tq;
+  d.scale_log2 = float(double(softmax_scale) * 1.4426950408889634);
+  return cuda_status(launch_window_attention(d, static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_get_device_status(void* ws, void* stream) {

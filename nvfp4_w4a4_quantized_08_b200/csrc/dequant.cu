@@ -12,69 +12,13 @@
 // the sink and window frames (171host.com LongLive 2.0 teardown, section 2.2)
 // back into contiguous bf16 K and V for attention.
 #include "common.cuh"
+#include "decode.cuh"
 #include "kernels.h"
 
 namespace nvfp4 {
 
 constexpr int kDqThreads = 256;
 constexpr int kDqUnroll = 2;
-
-// The 8 bf16 magnitudes of a block, as byte tables for prmt: lo0/lo1 hold the
-// low bytes of values 0..3 / 4..7, hi0/hi1 the high bytes.
-struct BlockLut {
-  uint32_t lo0, lo1, hi0, hi1;
-};
-
-__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ BlockLut make_lut(uint32_t sb, float s_t) {
-  const float s = e4m3_to_f32(sb);
-  // (v * s_b) is exact; one rounding for * s_t, one for bf16
-  const float f1 = __fmul_rn(__fmul_rn(0.5f, s), s_t);
-  const float f2 = __fmul_rn(s, s_t);
-  const float f3 = __fmul_rn(__fmul_rn(1.5f, s), s_t);
-  const float f4 = __fmul_rn(__fmul_rn(2.0f, s), s_t);
-  const float f5 = __fmul_rn(__fmul_rn(3.0f, s), s_t);
-  const float f6 = __fmul_rn(__fmul_rn(4.0f, s), s_t);
-  const float f7 = __fmul_rn(__fmul_rn(6.0f, s), s_t);
-  const uint32_t t01 = bf16x2_rn(0.0f, f1), t23 = bf16x2_rn(f2, f3);
-  const uint32_t t45 = bf16x2_rn(f4, f5), t67 = bf16x2_rn(f6, f7);
-  BlockLut l;
-  l.lo0 = prmt(t01, t23, 0x6420);
-  l.hi0 = prmt(t01, t23, 0x7531);
-  l.lo1 = prmt(t45, t67, 0x6420);
-  l.hi1 = prmt(t45, t67, 0x7531);
-  return l;
-}
-
-// 8 codes (nibble i of c = element i) -> 8 bf16 in four words.  Magnitudes
-// come from the block table (byte permutes indexed by the 3 magnitude bits);
-// the sign bits are gathered with one more permute per output word: se holds
-// the signs of the even elements at bit 7 of each byte, so those of the odd
-// elements, and the permute places element 2k's byte at byte 1 and element
-// 2k+1's at byte 3 of word k.
-__device__ __forceinline__ uint4 decode8(const BlockLut& l, uint32_t c) {
-  const uint32_t m = c & 0x77777777u;
-  const uint32_t mh = m >> 16;
-  uint4 o;
-  uint32_t lo4 = prmt(l.lo0, l.lo1, m), hi4 = prmt(l.hi0, l.hi1, m);
-  o.x = prmt(lo4, hi4, 0x5140);
-  o.y = prmt(lo4, hi4, 0x7362);
-  lo4 = prmt(l.lo0, l.lo1, mh);
-  hi4 = prmt(l.hi0, l.hi1, mh);
-  o.z = prmt(lo4, hi4, 0x5140);
-  o.w = prmt(lo4, hi4, 0x7362);
-  const uint32_t se = (c << 4) & 0x80808080u, so = c & 0x80808080u;
-  o.x |= prmt(se, so, 0x4000) & 0x80008000u;
-  o.y |= prmt(se, so, 0x5010) & 0x80008000u;
-  o.z |= prmt(se, so, 0x6020) & 0x80008000u;
-  o.w |= prmt(se, so, 0x7030) & 0x80008000u;
-  return o;
-}
 
 __device__ __forceinline__ uint32_t sf_mma_offset_dq(uint32_t row, uint32_t kb, uint32_t ktiles) {
   return ((row >> 7) * ktiles + (kb >> 2)) * 512u + (row & 31u) * 16u + ((row >> 5) & 3u) * 4u +

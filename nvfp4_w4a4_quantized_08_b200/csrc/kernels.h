@@ -61,6 +61,18 @@ struct LaunchKvDequant {
 };
 cudaError_t launch_kv_dequant(const LaunchKvDequant& d, cudaStream_t st);
 
+struct LaunchAttn {
+  const uint8_t *k_codes, *v_codes, *k_sf, *v_sf;
+  const float *k_st, *v_st;
+  const int32_t* slot_ids;  // host, n
+  int32_t n, tpf, heads;
+  const void* q;            // bf16
+  void* out;                // bf16
+  int64_t q_stride, out_stride, tq;
+  float scale_log2;         // softmax scale * log2(e)
+};
+cudaError_t launch_window_attention(const LaunchAttn& d, cudaStream_t st);
+
 struct LaunchGemm {
   const uint8_t* a_codes;
   const uint8_t* a_sf;

@@ -203,6 +203,29 @@ class KVCache:
                 "nvfp4_kv_dequant_window")
         return k_out, v_out
 
+    def window_attention(self, q: torch.Tensor, slot_ids: Sequence[int],
+                         scale: Optional[float] = None,
+                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """nvfp4_window_attention: softmax(scale q k^T) v over the listed slots,
+        read straight from the NVFP4 pools.  q: bf16 [tq, >= heads*head_dim]
+        (row stride a multiple of 8, e.g. the Q third of a QKV output) ->
+        bf16 [tq, heads*head_dim] (or `out`, same layout as q)."""
+        if q.dtype != torch.bfloat16 or q.dim() != 2 or q.stride(1) != 1:
+            raise ValueError("q must be a 2-D bf16 tensor with unit column stride")
+        if scale is None:
+            scale = self.head_dim ** -0.5
+        if out is None:
+            out = torch.empty(q.shape[0], self.heads * self.head_dim, dtype=torch.bfloat16,
+                              device=q.device)
+        n = len(slot_ids)
+        ids = (ctypes.c_int32 * n)(*slot_ids)
+        cs = self.c_struct()
+        N.check(N.lib().nvfp4_window_attention(ctypes.byref(cs), ids, n, q.data_ptr(), q.stride(0),
+                                               q.shape[0], float(scale), out.data_ptr(),
+                                               out.stride(0), _stream()),
+                "nvfp4_window_attention")
+        return out
+
 
 def device_status(ws: Optional[torch.Tensor] = None) -> int:
     """nvfp4_get_device_status: sync the current stream, read and clear the

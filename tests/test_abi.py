@@ -168,3 +168,29 @@ def test_no_gpu_means_arch_error_not_fallback(L):
     t = _tensor()
     assert L.nvfp4_quantize(FAKE, N.BF16, 256, 256, 256, ctypes.byref(t), None, None, FAKE, 256,
                             None) == N.ERR_ARCH
+
+
+def test_window_attention_rejects(L):
+    c = _cache()
+    f = L.nvfp4_window_attention
+    S = ctypes.c_int32 * 3
+    ids = S(0, 1, 2)
+    ok = (ids, 3, FAKE, 9216, 2640, 0.088, FAKE, 3072, None)
+    # argument checks run before any device query, so a call that passes them
+    # would reach the device: only failing combinations are exercised here
+    assert f(ctypes.byref(c), S(0, 1, 12), 3, *ok[2:]) == N.ERR_INVALID_ARG  # slot out of range
+    assert f(ctypes.byref(c), ids, 0, *ok[2:]) == N.ERR_INVALID_ARG
+    assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 2640, 0.0, FAKE, 3072,
+             None) == N.ERR_INVALID_ARG  # scale
+    assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 2640, float("nan"), FAKE, 3072,
+             None) == N.ERR_INVALID_ARG
+    assert f(ctypes.byref(c), ids, 3, FAKE, 3000, 2640, 0.088, FAKE, 3072,
+             None) == N.ERR_INVALID_ARG  # q stride below heads * head_dim
+    assert f(ctypes.byref(_cache(hd=64)), ids, 3, FAKE, 9216, 2640, 0.088, FAKE, 3072,
+             None) == N.ERR_UNSUPPORTED_SHAPE  # head_dim 128 only
+    assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 0, 0.088, FAKE, 3072,
+             None) == N.ERR_UNSUPPORTED_SHAPE  # tq
+    assert f(ctypes.byref(c), ids, 3, FAKE + 8, 9216, 2640, 0.088, FAKE, 3072,
+             None) == N.ERR_MISALIGNED
+    assert f(ctypes.byref(c), ids, 3, FAKE, 9220, 2640, 0.088, FAKE, 3072,
+             None) == N.ERR_MISALIGNED
