@@ -92,37 +92,58 @@ __global__ void __launch_bounds__(kAttThreads) window_attention_kernel(const Att
   const uint32_t n_tiles = (a.n_kv + kAttBK - 1) / kAttBK;
   for (uint32_t kt = 0; kt < n_tiles; ++kt) {
     __syncthreads();  // every warp is done with the previous tile
-    // ---- decode the K and V blocks of tokens [64 kt, 64 kt + 64) of head h
-    for (int i = threadIdx.x; i < 2 * kAttBK * kDimBlocks; i += kAttThreads) {
-      const int plane = i / (kAttBK * kDimBlocks);
-      const int r = i % (kAttBK * kDimBlocks);
-      const int tok = r / kDimBlocks, db = r % kDimBlocks;
-      const uint32_t j = kt * kAttBK + tok;
-      uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-      if (j < a.n_kv) {
+    // ---- decode the K and V blocks of tokens [64 kt, 64 kt + 64) of head h:
+    // 2 planes x 64 tokens x 8 blocks, 8 per thread, every pass's loads issued
+    // before any block is decoded.  K passes (it < 4): token threadIdx / 8 +
+    // 16 it, dim block threadIdx % 8 (a warp's 16-byte row stores spread over
+    // all banks).  V passes: token threadIdx % 64, dim block 2 (it - 4) +
+    // threadIdx / 64, so that a warp's transposed 16-bit stores hit 16
+    // consecutive words of one Vt row (dim-block-major lanes would put all 8
+    // blocks' rows, 16 x 36 words apart, in one bank).
+    {
+      auto tok_of = [](int it) {
+        return it < 4 ? int(threadIdx.x) / kDimBlocks + 16 * it : int(threadIdx.x) % kAttBK;
+      };
+      auto db_of = [](int it) {
+        return it < 4 ? int(threadIdx.x) % kDimBlocks : 2 * (it - 4) + int(threadIdx.x) / kAttBK;
+      };
+      uint2 c[8];
+      uint32_t sb[8];
+      float stv[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int plane = it / 4;
+        const int tok = tok_of(it), db = db_of(it);
+        const uint32_t j = min(kt * kAttBK + tok, a.n_kv - 1);  // past the end: reload, zeroed below
         const uint32_t pos = fast_div(a.tpf_div, j);  // position in the slot list
         const uint32_t local = j - pos * a.tpf;
         const size_t s = size_t(a.slots[pos]);
         const size_t blk = ((s * a.tpf + local) * a.heads + h) * kDimBlocks + db;
-        const uint8_t* codes = plane == 0 ? a.codes[0] : a.codes[1];
-        const uint8_t* sfp = plane == 0 ? a.sf[0] : a.sf[1];
-        const float* stp = plane == 0 ? a.st[0] : a.st[1];
-        const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes) + blk);
-        const BlockLut l = make_lut(__ldg(sfp + blk), __ldg(stp + s));
-        lo = decode8(l, c.x);
-        hi = decode8(l, c.y);
+        c[it] = __ldg(reinterpret_cast<const uint2*>(a.codes[plane]) + blk);
+        sb[it] = __ldg(a.sf[plane] + blk);
+        stv[it] = __ldg(a.st[plane] + s);
       }
-      if (plane == 0) {
-        uint4* dst = reinterpret_cast<uint4*>(Ks + tok * kLdK + 16 * db);
-        dst[0] = lo;
-        dst[1] = hi;
-      } else {
-        const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        uint16_t* col = Vt + (16 * db) * kLdV + tok;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          col[(2 * e) * kLdV] = uint16_t(w[e] & 0xFFFFu);
-          col[(2 * e + 1) * kLdV] = uint16_t(w[e] >> 16);
+      for (int it = 0; it < 8; ++it) {
+        const int tok = tok_of(it), db = db_of(it);
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+        if (kt * kAttBK + tok < a.n_kv) {
+          const BlockLut l = make_lut(sb[it], stv[it]);
+          lo = decode8(l, c[it].x);
+          hi = decode8(l, c[it].y);
+        }
+        if (it < 4) {
+          uint4* dst = reinterpret_cast<uint4*>(Ks + tok * kLdK + 16 * db);
+          dst[0] = lo;
+          dst[1] = hi;
+        } else {
+          const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          uint16_t* col = Vt + (16 * db) * kLdV + tok;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            col[(2 * e) * kLdV] = uint16_t(w[e] & 0xFFFFu);
+            col[(2 * e + 1) * kLdV] = uint16_t(w[e] >> 16);
+          }
         }
       }
     }
