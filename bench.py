@@ -9,7 +9,8 @@ stand-in -> out-proj GEMM -> quantize -> FFN-up GEMM (N=14336) with the GELU
 (tanh form) in its epilogue -> requantize the intermediate -> FFN-down GEMM;
 the down output feeds the next layer.  Attention, norms and residuals are not
 part of the NVFP4 path and are not run; the attention output is a fixed seeded
-tensor.  Weights are pre-quantized
+tensor; attention straight from the NVFP4 cache (nvfp4_window_attention) is
+timed separately on layer 0's window.  Weights are pre-quantized
 (outside the timed region).  The whole step is captured once as a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
