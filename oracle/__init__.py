@@ -15,7 +15,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
-from typing import Optional, Sequence, Tuple
+from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -326,3 +326,33 @@ def window_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
                                       _ptr(k), _ptr(v), n_kv, heads, hd, float(scale), _ptr(out),
                                       _ptr(E)), "window_attention")
     return out, E
+
+
+def sink_window_frames(chunks: Sequence[Tuple[int, bool]], global_sinks: int, shot_sinks: int,
+                       window: int) -> List[List[int]]:
+    """Frames each chunk of a multi-shot generation attends to, in frame order.
+
+    The two-level attention sinks (neurohive.io LongLive-2.0 article, inference
+    section; tailorednewshub.com article, "Sumidero de Atención Multi-Toma"):
+    the first `global_sinks` frames of the video stay for good, the first
+    `shot_sinks` frames of the current shot are re-bound at each cut; with the
+    local window of the last `window` frames, the chunk's own included
+    (171host.com teardown, section 2.2).  chunks: (n_frames, new_shot) in
+    generation order; the first chunk starts the first shot."""
+    out = []
+    f0 = 0
+    shot = 0
+    for n, new_shot in chunks:
+        f1 = f0 + n
+        if new_shot or f0 == 0:
+            shot = f0
+        frames = []
+        for f in range(f1):
+            in_global = f < global_sinks
+            in_shot = shot <= f < shot + shot_sinks
+            in_window = f >= f1 - window
+            if in_global or in_shot or in_window:
+                frames.append(f)
+        out.append(frames)
+        f0 = f1
+    return out
