@@ -276,6 +276,38 @@ NVFP4_API nvfp4_status nvfp4_window_attention(const nvfp4_kv_cache* cache, const
                                               int64_t tq, float softmax_scale, void* out,
                                               int64_t out_token_stride, void* stream);
 
+/* Slot planning for multi-shot generation (host only: no device work, no
+ * stream).  Each chunk of new frames attends to three sets of frames
+ * (neurohive.io LongLive-2.0 article, inference section on attention sinks;
+ * tailorednewshub.com LongLive-2.0 article, section "Sumidero de Atención
+ * Multi-Toma"; 171host.com teardown, section 2.2):
+ *   G: the first global_sinks frames of the video, kept for good;
+ *   H: the first shot_sinks frames of the current shot, re-bound at each cut;
+ *   L: the last `window` frames up to and including the chunk's own.
+ * A plan tracks which frame each of the cache's n_slots slots holds.
+ *   create:  n_slots >= global_sinks + shot_sinks + window (enough for any
+ *            G u H u L), n_slots <= NVFP4_KV_MAX_WINDOW_SLOTS, window >= 1;
+ *            NULL on invalid arguments or allocation failure.
+ *   next:    plan the next chunk of n_frames frames (1..8, <= window);
+ *            new_shot != 0 when the chunk starts a new shot (the first chunk
+ *            always does).  Frees every slot whose frame is outside the
+ *            chunk's G u H u L (never attended again), writes the lowest free
+ *            slots for the chunk's frames to dst_slots[n_frames] (for
+ *            nvfp4_kv_quant_chunk), and the slots of G u H u L in frame order
+ *            to window_slots (capacity n_slots; count in *n_window) for
+ *            nvfp4_kv_dequant_window / nvfp4_window_attention.
+ *            Errors: INVALID_ARG (the plan is unchanged).
+ *   frame_of_slot: the frame a slot holds, -1 if free or out of range.
+ * The caller owns the plan (destroy frees it); a plan is not thread-safe. */
+typedef struct nvfp4_sink_plan nvfp4_sink_plan;
+NVFP4_API nvfp4_sink_plan* nvfp4_sink_plan_create(int32_t n_slots, int32_t global_sinks,
+                                                  int32_t shot_sinks, int32_t window);
+NVFP4_API void nvfp4_sink_plan_destroy(nvfp4_sink_plan* plan);
+NVFP4_API nvfp4_status nvfp4_sink_plan_next(nvfp4_sink_plan* plan, int32_t n_frames,
+                                            int32_t new_shot, int32_t* dst_slots,
+                                            int32_t* window_slots, int32_t* n_window);
+NVFP4_API int64_t nvfp4_sink_plan_frame_of_slot(const nvfp4_sink_plan* plan, int32_t slot);
+
 /* Size of the library-owned scratch array behind nvfp4_quantize_noalloc. */
 #define NVFP4_NOALLOC_SCRATCH_BYTES 256
 

@@ -9,5 +9,5 @@ refuses any device that is not sm_100.
 from ._native import (ACT_GELU_TANH, ACT_NONE, BF16, FP32, KV_MAX_CHUNK_FRAMES,  # noqa: F401
                       KV_MAX_WINDOW_SLOTS, SCALE_FOUR_OVER_SIX, SCALE_ONTO_6, SF_MMA128x4,
                       SF_ROWMAJOR, NVFP4Error)
-from .ops import (KVCache, NVFP4Tensor, codes_bytes, dequantize, device_status, empty,  # noqa: F401
-                  gemm, quantize, set_wait_limit_ns, sf_bytes, workspace)
+from .ops import (KVCache, NVFP4Tensor, SinkPlan, codes_bytes, dequantize,  # noqa: F401
+                  device_status, empty, gemm, quantize, set_wait_limit_ns, sf_bytes, workspace)

@@ -38,7 +38,8 @@ EXPORTS = (
     "nvfp4_codes_bytes", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
     "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_quant_chunk", "nvfp4_kv_dequant_window",
     "nvfp4_get_device_status", "nvfp4_set_wait_limit_ns", "nvfp4_status_string",
-    "nvfp4_quantize_noalloc", "nvfp4_window_attention",
+    "nvfp4_quantize_noalloc", "nvfp4_window_attention", "nvfp4_sink_plan_create",
+    "nvfp4_sink_plan_destroy", "nvfp4_sink_plan_next", "nvfp4_sink_plan_frame_of_slot",
 )
 
 
@@ -95,6 +96,16 @@ def lib() -> ctypes.CDLL:
                                              vp, vp, vp, sz, vp]
         L.nvfp4_kv_dequant_window.restype = i32
         L.nvfp4_kv_dequant_window.argtypes = [KP, ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
+        L.nvfp4_sink_plan_create.restype = vp
+        L.nvfp4_sink_plan_create.argtypes = [i32, i32, i32, i32]
+        L.nvfp4_sink_plan_destroy.restype = None
+        L.nvfp4_sink_plan_destroy.argtypes = [vp]
+        L.nvfp4_sink_plan_next.restype = i32
+        L.nvfp4_sink_plan_next.argtypes = [vp, i32, i32, ctypes.POINTER(ctypes.c_int32),
+                                           ctypes.POINTER(ctypes.c_int32),
+                                           ctypes.POINTER(ctypes.c_int32)]
+        L.nvfp4_sink_plan_frame_of_slot.restype = i64
+        L.nvfp4_sink_plan_frame_of_slot.argtypes = [vp, i32]
         L.nvfp4_window_attention.restype = i32
         L.nvfp4_window_attention.argtypes = [KP, ctypes.POINTER(ctypes.c_int32), i32, vp, i64,
                                              i64, ctypes.c_float, vp, i64, vp]

@@ -8,7 +8,7 @@ from __future__ import annotations
 
 import ctypes
 from dataclasses import dataclass
-from typing import Dict, Optional, Sequence, Tuple
+from typing import Dict, List, Optional, Sequence, Tuple
 
 import torch
 
@@ -225,6 +225,39 @@ class KVCache:
                                                out.stride(0), _stream()),
                 "nvfp4_window_attention")
         return out
+
+
+class SinkPlan:
+    """nvfp4_sink_plan: host-side slot planning under the two-level attention
+    sinks (global sinks kept for good, shot sinks re-bound at cuts, a local
+    window).  next() -> (dst_slots for KVCache.quant_chunk, window slot list
+    for KVCache.dequant_window / window_attention)."""
+
+    def __init__(self, n_slots: int, global_sinks: int = 3, shot_sinks: int = 3,
+                 window: int = 9):
+        self.n_slots = n_slots
+        self._h = N.lib().nvfp4_sink_plan_create(n_slots, global_sinks, shot_sinks, window)
+        if not self._h:
+            raise N.NVFP4Error(N.ERR_INVALID_ARG, "nvfp4_sink_plan_create")
+
+    def next(self, n_frames: int, new_shot: bool = False) -> Tuple[List[int], List[int]]:
+        dst = (ctypes.c_int32 * max(1, n_frames))()
+        win = (ctypes.c_int32 * self.n_slots)()
+        n = ctypes.c_int32(0)
+        N.check(N.lib().nvfp4_sink_plan_next(self._h, n_frames, int(bool(new_shot)), dst, win,
+                                             ctypes.byref(n)), "nvfp4_sink_plan_next")
+        return list(dst[:n_frames]), list(win[:n.value])
+
+    def frame_of_slot(self, slot: int) -> int:
+        return int(N.lib().nvfp4_sink_plan_frame_of_slot(self._h, slot))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            N.lib().nvfp4_sink_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
 
 
 def device_status(ws: Optional[torch.Tensor] = None) -> int:
