@@ -290,7 +290,9 @@ class CpuSample:
         o.gemm(o.quantize(self.x), self.wq[0])
         y, _ = o.gemm(o.quantize(self.attn), self.wq[1])
         u, _ = o.gemm(o.quantize(to_bf16_bits(y)), self.wq[2])
-        o.gemm(o.quantize(to_bf16_bits(u)), self.wq[3])
+        # the FFN GELU on the bf16 up-projection output, as the GPU step computes it
+        u16 = (to_bf16_bits(u).astype(np.uint32) << 16).view(np.float32)
+        o.gemm(o.quantize(to_bf16_bits(o.gelu_tanh(u16))), self.wq[3])
         t_rows = time.perf_counter() - t0
         t0 = time.perf_counter()
         ck, sk, tk = o.kv_quant_chunk(self.kv, 1, TPF, wl.HEADS, wl.HEAD_DIM)
@@ -301,7 +303,8 @@ class CpuSample:
         flops = self.rows * GEMM_FLOPS_LAYER / M
         kv_bytes = 2 * 2 * KV_ELEMS_FRAME * Q_BYTES_PER_ELEM
         desc = (f"CPU oracle, {self.rows} of {M} token rows through one layer (4 activation "
-                f"quantizations + 4 FP64 GEMMs: {flops / 1e9:.2f} GFLOP in {t_rows:.2f} s) and "
+                f"quantizations, the FFN GELU + 4 FP64 GEMMs: {flops / 1e9:.2f} GFLOP in "
+                f"{t_rows:.2f} s) and "
                 f"the K+V codec of one 880-token frame ({kv_bytes / 1e6:.1f} MB in {t_kv:.2f} s)")
         return {"tflops": flops / t_rows / 1e12, "kv_gbs": kv_bytes / t_kv / 1e9,
                 "cores": self.cores, "sample": desc, "seconds": t_rows + t_kv}
