@@ -210,13 +210,17 @@ class KVCache:
         read straight from the NVFP4 pools.  q: bf16 [tq, >= heads*head_dim]
         (row stride a multiple of 8, e.g. the Q third of a QKV output) ->
         bf16 [tq, heads*head_dim] (or `out`, same layout as q)."""
-        if q.dtype != torch.bfloat16 or q.dim() != 2 or q.stride(1) != 1:
-            raise ValueError("q must be a 2-D bf16 tensor with unit column stride")
+        width = self.heads * self.head_dim
+        if q.dtype != torch.bfloat16 or q.dim() != 2 or q.stride(1) != 1 or q.shape[1] < width:
+            raise ValueError(f"q must be a 2-D bf16 tensor of at least {width} unit-stride columns")
         if scale is None:
             scale = self.head_dim ** -0.5
         if out is None:
-            out = torch.empty(q.shape[0], self.heads * self.head_dim, dtype=torch.bfloat16,
-                              device=q.device)
+            out = torch.empty(q.shape[0], width, dtype=torch.bfloat16, device=q.device)
+        elif (out.dtype != torch.bfloat16 or out.dim() != 2 or out.stride(1) != 1 or
+              out.shape[0] != q.shape[0] or out.shape[1] < width):
+            raise ValueError(f"out must be a 2-D bf16 tensor of {q.shape[0]} rows and at least "
+                             f"{width} unit-stride columns")
         n = len(slot_ids)
         ids = (ctypes.c_int32 * n)(*slot_ids)
         cs = self.c_struct()
@@ -257,7 +261,10 @@ class SinkPlan:
             self._h = None
 
     def __del__(self):
-        self.close()
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown: the library may be gone already
+            pass
 
 
 def device_status(ws: Optional[torch.Tensor] = None) -> int:

@@ -194,3 +194,18 @@ def test_window_attention_rejects(L):
              None) == N.ERR_MISALIGNED
     assert f(ctypes.byref(c), ids, 3, FAKE, 9220, 2640, 0.088, FAKE, 3072,
              None) == N.ERR_MISALIGNED
+
+
+def test_sink_plan_null_and_bad_arguments(L):
+    S = ctypes.c_int32 * 16
+    n = ctypes.c_int32(0)
+    assert L.nvfp4_sink_plan_next(None, 3, 0, S(), S(), ctypes.byref(n)) == N.ERR_INVALID_ARG
+    assert not L.nvfp4_sink_plan_create(15, -1, 3, 9)
+    assert not L.nvfp4_sink_plan_create(15, 3, 3, 0)
+    h = L.nvfp4_sink_plan_create(15, 3, 3, 9)
+    assert h
+    assert L.nvfp4_sink_plan_next(h, 3, 0, None, S(), ctypes.byref(n)) == N.ERR_INVALID_ARG
+    assert L.nvfp4_sink_plan_frame_of_slot(None, 0) == -1
+    assert L.nvfp4_sink_plan_frame_of_slot(h, 0) == -1  # nothing planned yet
+    L.nvfp4_sink_plan_destroy(h)
+    L.nvfp4_sink_plan_destroy(None)  # a no-op
