@@ -30,15 +30,18 @@ class OracleError(RuntimeError):
     pass
 
 
+# gcc flags of the oracle: IEEE binary32 with no contraction, OpenMP on outer loops
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+          "-fno-fast-math", "-fexcess-precision=standard"]
+
+
 def build(force: bool = False) -> str:
     """Compile liboracle.so with gcc (IEEE binary32, no contraction, OpenMP)."""
     if (not force and os.path.exists(_LIB)
             and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
         return _LIB
     tmp = _LIB + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-           "-ffp-contract=off", "-fno-fast-math", "-fexcess-precision=standard",
-           "-o", tmp, _SRC, "-lm"]
+    cmd = ["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, _LIB)
     return _LIB

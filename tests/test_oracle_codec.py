@@ -246,3 +246,92 @@ def test_kv_window_is_per_slot_dequant(orc):
         np.testing.assert_array_equal(out[i * tpf:(i + 1) * tpf].reshape(tpf * heads, hd), ref)
     with pytest.raises(orc.OracleError):
         orc.kv_dequant_window(pool_c, pool_s, pool_t, [6], tpf, heads, hd)
+
+
+# ------------------------------------------------------------------ evaluation order
+# The recipe fixes one binary32 rounding per written step: r = amax_b / RN(6 s_t),
+# y = x / RN(s_b s_t), f = RN(v s_b) * s_t.  Random inputs almost never tell these
+# apart from other orders, so these pins search (numpy binary32, fixed seeds) for
+# inputs where another order gives a different byte, and check the oracle there.
+def _e4m3(r):
+    return np.minimum(np.asarray(r, F32), F32(448.0)).astype(ml_dtypes.float8_e4m3fn) \
+        .view(np.uint8)
+
+
+def _e2m1(y):
+    return np.clip(np.asarray(y, F32), -6, 6).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+
+
+def _nudge(x, k):
+    """x moved by k binary32 ulps (elementwise)."""
+    out = np.asarray(x, F32).copy()
+    for _ in range(abs(int(k))):
+        out = np.nextafter(out, F32(np.inf) if k > 0 else F32(0)).astype(F32)
+    return out
+
+
+def test_block_scale_evaluation_order(orc):
+    rng = np.random.default_rng(21)
+    vals = np.array([float(np.array(c, np.uint8).view(ml_dtypes.float8_e4m3fn)) for c in
+                     range(0x7F)])
+    mids = (vals[:-1] + vals[1:]) / 2          # E4M3 rounding boundaries
+    n = 20000
+    s_t = rng.uniform(1e-4, 1e-1, n).astype(F32)
+    six_st = F32(6.0) * s_t
+    amax = (mids[rng.integers(1, len(mids), n)] * six_st).astype(F32)
+    amax = np.concatenate([_nudge(amax[i::5], k) for i, k in enumerate(range(-2, 3))])
+    s_t = np.concatenate([s_t[i::5] for i in range(5)])
+    right = _e4m3(amax / (F32(6.0) * s_t))
+    other = np.stack([_e4m3((amax / s_t) / F32(6.0)), _e4m3(amax / F32(6.0) / s_t),
+                      _e4m3(amax * (F32(1.0) / (F32(6.0) * s_t)))])
+    sens = np.nonzero((other != right).any(axis=0))[0]
+    assert len(sens) >= 20
+    for i in sens[:400]:
+        assert orc.block_scale(float(amax[i]), float(s_t[i])) == int(right[i]), i
+
+
+def test_element_code_evaluation_order(orc):
+    rng = np.random.default_rng(22)
+    n = 20000
+    s_t = rng.uniform(1e-4, 1e-1, n).astype(F32)
+    sb = rng.integers(0x20, 0x7E, n).astype(np.uint8)
+    sbv = sb.view(ml_dtypes.float8_e4m3fn).astype(F32)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], F32)
+    d = sbv * s_t
+    x = (ties[rng.integers(0, len(ties), n)] * d).astype(F32)
+    x = np.concatenate([_nudge(x[i::3], k) for i, k in enumerate(range(-1, 2))])
+    s_t = np.concatenate([s_t[i::3] for i in range(3)])
+    sb = np.concatenate([sb[i::3] for i in range(3)])
+    sbv = sb.view(ml_dtypes.float8_e4m3fn).astype(F32)
+    right = _e2m1(x / (sbv * s_t))
+    other = np.stack([_e2m1((x / sbv) / s_t), _e2m1((x / s_t) / sbv),
+                      _e2m1(x * (F32(1.0) / (sbv * s_t)))])
+    sens = np.nonzero((other != right).any(axis=0))[0]
+    assert len(sens) >= 20
+    for i in sens[:400]:
+        assert orc.element_code(float(x[i]), int(sb[i]), float(s_t[i])) == int(right[i]), i
+
+
+def test_dequant_evaluation_order(orc):
+    """(v s_b) s_t versus v (s_b s_t): only v in {1.5, 3, 6} can tell them
+    apart, and only next to a bf16 rounding midpoint; aim s_t at midpoints."""
+    rng = np.random.default_rng(23)
+    n = 30000
+    code = rng.choice([3, 5, 7], n)                       # v = 1.5, 3, 6
+    v = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], F32)[code]
+    sb = rng.integers(0x20, 0x7E, n).astype(np.uint8)
+    sbv = sb.view(ml_dtypes.float8_e4m3fn).astype(F32)
+    # bf16 midpoints m = (2k + 1) 2^(e-8), exact in binary32
+    mid = ((2 * rng.integers(128, 256, n) + 1) * np.exp2(rng.integers(-20, 4, n) - 8.0))
+    s_t = (mid / (v.astype(np.float64) * sbv.astype(np.float64))).astype(F32)
+    s_t = np.concatenate([_nudge(s_t[i::5], k) for i, k in enumerate(range(-2, 3))])
+    code = np.concatenate([code[i::5] for i in range(5)])
+    sb = np.concatenate([sb[i::5] for i in range(5)])
+    v = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], F32)[code]
+    sbv = sb.view(ml_dtypes.float8_e4m3fn).astype(F32)
+    right = bf16_bits((v * sbv) * s_t)
+    other = bf16_bits(v * (sbv * s_t))
+    sens = np.nonzero(other != right)[0]
+    assert len(sens) >= 20
+    for i in sens[:400]:
+        assert orc.dequant_elem(int(code[i]), int(sb[i]), float(s_t[i])) == int(right[i]), i

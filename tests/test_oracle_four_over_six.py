@@ -131,3 +131,25 @@ def test_kv_chunk_rule_never_increases_block_error(orc):
     # the codes under either rule are the plain recipe's codes for that block scale
     for b in range(0, x.shape[0], 7):
         np.testing.assert_array_equal(q1[b], _codes(x[b], int(s1.reshape(-1)[b]), st))
+
+
+def test_exact_tie_keeps_six(orc):
+    """A block coded without error by both scales: with s_t = 1/16 and maximum
+    0.75, onto 6 gives s_b = 2 (grid {0, .5, 1, 1.5, 2, 3, 4, 6} / 8) and onto 4
+    gives s_b = 3 (grid {0, .75, 1.5, 2.25, 3, 4.5, 6, 9} / 16); the values
+    0.75, 0.375 and 0.1875 lie on both, so both squared errors are exactly 0
+    and the rule keeps 6."""
+    block = np.zeros(16, np.float32)
+    block[[0, 3, 7, 12]] = [0.75, 0.375, -0.1875, 0.375]
+    s_t = 1.0 / 16
+    six = orc.block_scale_rule(block, s_t, 0)
+    assert orc.e4m3_value(six) == 2.0
+    assert orc.block_scale_rule(block, s_t, 1) == six
+    # the onto-4 scale really is different and exact too
+    s4 = int(np.array(0.75 / (4 * s_t), np.float32).astype(ml_dtypes.float8_e4m3fn)
+             .view(np.uint8))
+    assert orc.e4m3_value(s4) == 3.0
+    for x in block:
+        for s in (2.0, 3.0):
+            q = abs(float(x)) / (s * s_t)
+            assert q in (0, 0.5, 1, 1.5, 2, 3, 4, 6)
