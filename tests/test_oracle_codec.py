@@ -85,6 +85,10 @@ def test_tensor_scale_is_amax_over_2688(orc):
     amax, st = orc.tensor_scale(x)
     assert amax == np.max(np.abs(x))
     assert F32(st) == F32(amax) / F32(6 * 448)
+    # the largest magnitude negative: amax is a magnitude
+    x[7, 11] = -4 * np.max(np.abs(x))
+    amax, st = orc.tensor_scale(x)
+    assert amax == -x[7, 11] and F32(st) == F32(-x[7, 11]) / F32(6 * 448)
 
 
 # ------------------------------------------------------------------ round trips

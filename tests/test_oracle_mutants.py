@@ -69,6 +69,28 @@ MUTANTS = [
      "const uint16_t* kj = k + (j * heads) * (int64_t)head_dim;", ["test_oracle_attention.py"]),
     ("attention magnitude sum signed", "e[d] += p * fabs(x);", "e[d] += p * x;",
      ["test_oracle_attention.py"]),
+    ("tensor amax ignores the sign", "else amax = fmaxf(amax, fabsf(v));",
+     "else amax = fmaxf(amax, v);", CODEC),
+    ("E4M3 saturates to the NaN byte", "if (x >= 448.0) return 0x7E | (signbit(r) ? 0x80 : 0);",
+     "if (x >= 448.0) return 0x7F | (signbit(r) ? 0x80 : 0);", FORMATS),
+    ("exact dequant uses the next block's scale",
+     "out[i * cols + j] = orc_e2m1_value(q) * orc_e4m3_value(sf[i * nkb + j / 16]) * (double)s_t;",
+     "out[i * cols + j] = orc_e2m1_value(q) * orc_e4m3_value(sf[i * nkb + (j / 16 + 1) % nkb]) "
+     "* (double)s_t;", GEMM),
+    ("window rebuild takes the list position's tensor scale",
+     "pool_sf + s * frame_sf, pool_st[s], rows,", "pool_sf + s * frame_sf, pool_st[i], rows,",
+     CODEC),
+]
+
+# the same for the oracle's Python functions: (mistake, function, text, planted text, pins)
+PY_MUTANTS = [
+    ("sink window one frame short", "sink_window_frames", "in_window = f >= f1 - window",
+     "in_window = f > f1 - window", ["test_oracle_sink_plan.py"]),
+    ("shot sinks never re-bound", "sink_window_frames", "if new_shot or f0 == 0:",
+     "if f0 == 0:", ["test_oracle_sink_plan.py"]),
+    ("shot sinks one frame too many", "sink_window_frames",
+     "in_shot = shot <= f < shot + shot_sinks", "in_shot = shot <= f <= shot + shot_sinks",
+     ["test_oracle_sink_plan.py"]),
 ]
 
 
@@ -85,6 +107,25 @@ def test_pins_reject_planted_mistake(tmp_path, mistake, old, new, files):
     paths = [os.path.join(ROOT, "tests", f) for f in files]
     code = (f"import sys; sys.path.insert(0, {ROOT!r}); import oracle; "
             f"oracle._LIB = {mutant_so!r}; oracle.build = lambda force=False: oracle._LIB; "
+            f"import pytest; sys.exit(pytest.main(['-q', '-x', '-p', 'no:cacheprovider', "
+            f"'-m', 'not gpu', *{paths!r}]))")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 1 and " failed" in r.stdout, (
+        f"{mistake}: the pins did not catch it (exit {r.returncode})\n{r.stdout[-1500:]}")
+
+
+@pytest.mark.parametrize("mistake,func,old,new,files", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_pins_reject_planted_mistake_python(mistake, func, old, new, files):
+    sys.path.insert(0, ROOT)
+    import inspect
+
+    import oracle
+    assert inspect.getsource(getattr(oracle, func)).count(old) == 1, mistake
+    paths = [os.path.join(ROOT, "tests", f) for f in files]
+    code = (f"import sys, inspect; sys.path.insert(0, {ROOT!r}); import oracle; "
+            f"src = inspect.getsource(oracle.{func}).replace({old!r}, {new!r}); "
+            f"exec(src, oracle.__dict__); "
             f"import pytest; sys.exit(pytest.main(['-q', '-x', '-p', 'no:cacheprovider', "
             f"'-m', 'not gpu', *{paths!r}]))")
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
