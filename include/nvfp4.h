@@ -14,6 +14,11 @@
  *     rebuilt to bf16 for windowed attention (hyper.ai LongLive-2.0 summary,
  *     section "方法" (Method), second paragraph), over a window of 9 local plus
  *     3 sink frames (171host.com LongLive 2.0 teardown, section 2.2).
+ *   - Around them: the FFN's GELU in the GEMM epilogue, windowed attention that
+ *     reads the NVFP4 cache directly, and host-side slot planning under the
+ *     two-level (global and per-shot) attention sinks of multi-shot generation
+ *     (neurohive.io article, inference section; tailorednewshub.com article,
+ *     section "Sumidero de Atención Multi-Toma").
  *
  * Quantization recipe (the pages name the format only; this library fixes):
  *   s_t = amax(|x|) / 2688                          (2688 = 6 * 448)
@@ -27,9 +32,10 @@
  *     "host" pointers are ordinary host memory read before the call returns.
  *   - The caller owns and allocates every buffer; the library allocates no
  *     device memory.  It caches per-device kernel attributes only.
- *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
- *     default stream).  Argument checks happen on the host, before any launch,
- *     and a rejected call launches nothing.
+ *   - Every call that takes a `stream` is asynchronous on it (a cudaStream_t;
+ *     NULL = the legacy default stream).  Argument checks happen on the host,
+ *     before any launch, and a rejected call launches nothing.  The sink-plan
+ *     calls are host-only and synchronous.
  *   - A launch failure returns NVFP4_ERR_CUDA.  Errors found on the device (a
  *     bounded wait that ran out, a tensor scale outside the recipe's domain) are
  *     recorded in the workspace status word and returned by
