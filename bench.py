@@ -39,17 +39,10 @@ sys.path.insert(0, ROOT)
 import nvfp4_w4a4_quantized_08_b200 as nv  # noqa: E402
 from nvfp4_w4a4_quantized_08_b200 import workloads as wl  # noqa: E402
 
-M = wl.CHUNK_TOKENS          # 2640
-D = wl.DIM                   # 3072
-F = wl.FFN                   # 14336
-QKV = wl.QKV_N               # 9216
-TPF = wl.TOKENS_PER_FRAME    # 880
-NEW_FRAMES = wl.CHUNK_FRAMES  # 3
-WINDOW = wl.SINK_FRAMES + wl.WINDOW_FRAMES  # 12
-POOL = WINDOW + NEW_FRAMES   # 15 slots per layer
+from nvfp4_w4a4_quantized_08_b200.dit_step import (D, F, GEMM_FLOPS_LAYER, GEMM_SHAPES,  # noqa: E402
+                                                   M, NEW_FRAMES, POOL, QKV, TPF, WINDOW,
+                                                   DiTStep)
 
-GEMM_SHAPES = {"qkv": (M, QKV, D), "out": (M, D, D), "up": (M, F, D), "down": (M, D, F)}
-GEMM_FLOPS_LAYER = sum(2 * m * n * k for (m, n, k) in GEMM_SHAPES.values())
 Q_BYTES_PER_ELEM = 2 + 0.5625     # bf16 in, 4-bit code + 1/16 E4M3 scale out
 KV_ELEMS_FRAME = TPF * wl.HEADS * wl.HEAD_DIM
 CODEC_BYTES = {
@@ -81,99 +74,6 @@ def max_over_ranks(value: float, dist, device) -> float:
 def job_throughput(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
     """Whole-job TFLOP/s: every rank runs its own step (weak scaling)."""
     return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
-
-
-# ---------------------------------------------------------------- model state
-class Step:
-    """Device state of the denoise step and the per-layer launch sequence."""
-
-    def __init__(self, layers: int, device):
-        self.layers = layers
-        self.dev = device
-        self.w = []       # per layer: (qkv, out, up, down) NVFP4 weights
-        self.cache = []
-        for l in range(layers):
-            ws_bf16 = wl.layer_weights_cuda(l, device=device)
-            self.w.append([nv.quantize(t) for t in ws_bf16])
-            del ws_bf16
-            c = nv.KVCache(POOL, TPF, wl.HEADS, wl.HEAD_DIM, device=device)
-            # prefill the 12 cached frames (sinks + window) with seeded K/V
-            kv = wl.kv_tensor_cuda(seed=l, tokens=WINDOW * TPF, device=device)
-            for f0 in (0, 8):
-                nf = min(8, WINDOW - f0)
-                sl = kv[f0 * TPF:(f0 + nf) * TPF]
-                c.quant_chunk(sl, sl, list(range(f0, f0 + nf)))
-            self.cache.append(c)
-        torch.cuda.synchronize()
-        self.x_in = wl.activations(c=5, i=0).to(device)          # step input
-        self.attn = wl.randn((M, D), 5, 1).to(device)           # attention-output stand-in
-        self.qkv_out = torch.empty(M, QKV, dtype=torch.bfloat16, device=device)
-        self.o_out = torch.empty(M, D, dtype=torch.bfloat16, device=device)
-        self.up_out = torch.empty(M, F, dtype=torch.bfloat16, device=device)
-        self.down_out = [torch.empty(M, D, dtype=torch.bfloat16, device=device) for _ in range(2)]
-        self.k_win = torch.empty(WINDOW * TPF, wl.HEADS, wl.HEAD_DIM, dtype=torch.bfloat16,
-                                 device=device)
-        self.v_win = torch.empty_like(self.k_win)
-        self.qa = nv.empty(M, D, device=device)
-        self.qf = nv.empty(M, F, device=device)
-        self.ws = nv.workspace(device)
-        # max|C| words handed from a GEMM epilogue to the quantization of its
-        # output: [0] down -> next layer's input, [1] out-proj, [2] FFN up,
-        # [3..5] the Q, K, V thirds of the QKV projection (K, V -> KV chunk)
-        self.amax = torch.zeros(6, dtype=torch.float32, device=device)
-        self.new_slots = list(range(WINDOW, POOL))
-        self.window = list(range(wl.SINK_FRAMES)) + \
-            list(range(wl.SINK_FRAMES + NEW_FRAMES, WINDOW)) + self.new_slots
-        assert len(self.window) == WINDOW
-
-    def output(self) -> torch.Tensor:
-        return self.down_out[(self.layers - 1) % 2]
-
-    def run(self, mark=None):
-        """Enqueue one step on the current stream.  `mark(name)` (optional) is
-        called before each launch group and once at the end with None."""
-        mk = mark or (lambda name: None)
-        x = self.x_in
-        a_x, a_o, a_u = self.amax[0:1], self.amax[1:2], self.amax[2:3]
-        for l in range(self.layers):
-            wq, wo, wu, wd = self.w[l]
-            mk("quant_act")
-            # layer 0's input has no producer in the step: it takes the amax pass
-            nv.quantize(x, out=self.qa, ws=self.ws, amax_in=a_x if l > 0 else None)
-            mk("gemm_qkv")
-            nv.gemm(self.qa, wq, out=self.qkv_out, ws=self.ws, c_amax=self.amax[3:6],
-                    c_amax_cols=D)
-            mk("kv_quant")
-            self.cache[l].quant_chunk(self.qkv_out[:, D:2 * D], self.qkv_out[:, 2 * D:],
-                                      self.new_slots, ws=self.ws, k_amax_in=self.amax[4:5],
-                                      v_amax_in=self.amax[5:6])
-            mk("kv_dequant")
-            self.cache[l].dequant_window(self.window, self.k_win, self.v_win)
-            mk("quant_act")
-            nv.quantize(self.attn, out=self.qa, ws=self.ws)
-            mk("gemm_out")
-            nv.gemm(self.qa, wo, out=self.o_out, ws=self.ws, c_amax=a_o)
-            mk("quant_act")
-            nv.quantize(self.o_out, out=self.qa, ws=self.ws, amax_in=a_o)
-            mk("gemm_up")
-            # FFN up-projection with its GELU in the epilogue; the stored GELU
-            # output's amax feeds the intermediate requantization
-            nv.gemm(self.qa, wu, out=self.up_out, ws=self.ws, c_amax=a_u,
-                    act=nv.ACT_GELU_TANH)
-            mk("requant_ffn")
-            nv.quantize(self.up_out, out=self.qf, ws=self.ws, amax_in=a_u)
-            mk("gemm_down")
-            x = self.down_out[l % 2]
-            # the last layer's output is not quantized within the step
-            last = l == self.layers - 1
-            nv.gemm(self.qf, wd, out=x, ws=self.ws, c_amax=None if last else a_x)
-        mk(None)
-
-    # kernels launched per step: a quantize with its own amax pass 2 (layer 0's
-    # input, the attention output), one fed by a GEMM's c_amax 1, gemm 1,
-    # kv_quant 1 (its amax comes from the QKV GEMM), kv_dequant 1
-    def launches_per_step(self) -> int:
-        return self.layers * (2 + 1 + 1 + 1 + 4 * 1 + 1 + 1) + 1
 
 
 # ---------------------------------------------------------------- clocks
@@ -259,10 +159,10 @@ class CpuSample:
     weights pre-quantized by the oracle once, not timed), and the K + V codec
     (quantize + dequantize) of one latent frame."""
 
-    def __init__(self, rows: int = 16, seed_layer: int = 0):
+    def __init__(self, rows: int = 16, seed_layer: int = 0, threads: int = 0):
         import oracle
         self.oracle = oracle
-        self.cores = oracle.set_threads(0)
+        self.cores = oracle.set_threads(threads)
         self.rows = rows
         if torch.cuda.is_available():
             wts = [t.cpu() for t in wl.layer_weights_cuda(seed_layer, device="cuda")]
@@ -357,7 +257,7 @@ def config_block(args):
 ATTN_FLOPS = 4 * M * WINDOW * TPF * wl.HEAD_DIM * wl.HEADS  # QK^T and PV, one layer
 
 
-def time_window_attention(step: "Step", dev, reps: int = 10) -> float:
+def time_window_attention(step: DiTStep, dev, reps: int = 10) -> float:
     """Device ms of one nvfp4_window_attention: the chunk's 2640 queries (the Q
     third of the QKV output) over layer 0's 12-slot window read from the NVFP4
     pools, graph-replayed."""
@@ -386,7 +286,7 @@ def time_window_attention(step: "Step", dev, reps: int = 10) -> float:
     return e0.elapsed_time(e1) / reps
 
 
-def time_kv_four_over_six(step: "Step", dev, reps: int = 20) -> float:
+def time_kv_four_over_six(step: DiTStep, dev, reps: int = 20) -> float:
     """Device ms of one nvfp4_kv_quant_chunk (3 frames of K and V read from a
     QKV output, amax pass included) with the Four Over Six scale rule."""
     cache = nv.KVCache(POOL, TPF, wl.HEADS, wl.HEAD_DIM, device=dev,
@@ -414,6 +314,247 @@ def time_kv_four_over_six(step: "Step", dev, reps: int = 20) -> float:
     return e0.elapsed_time(e1) / reps
 
 
+class L2Flush:
+    """Writes a buffer twice the size of L2 so the next timed call starts with
+    its inputs in HBM only."""
+
+    def __init__(self, dev):
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.buf = torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def time_flushed(fn, flush, reps: int = 20, warmup: int = 3) -> float:
+    """Median device ms of fn() over `reps` calls, L2 flushed before each one;
+    CUDA events on the launching stream bracket fn() alone."""
+    cur = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(reps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        fn()
+        e1.record(cur)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def time_configs(dev, peaks) -> dict:
+    """The four single-call workloads, each timed on its own with L2 flushed
+    before every call (median of 20):
+      tiny: A and B fp32 256x256 with 2% x50 outliers -- quantize (amax pass
+        included), dequantize, FP4 GEMM 256^3 (fp32 out): microseconds;
+      qkv: activation quantization (amax pass included) + QKV GEMM
+        2640x9216x3072 (bf16 out): TFLOP/s of the pair;
+      ffn: quantize X, FFN-up 2640x14336x3072 with the GELU epilogue and its
+        amax hand-off, requantize the intermediate, FFN-down 2640x3072x14336:
+        TFLOP/s of the chain;
+      kv: K and V [10560, 24, 128] quantized in chunks of 8 and 4 frames (amax
+        pass included), then the 12-slot window rebuilt to bf16: GB/s."""
+    flush = L2Flush(dev)
+    ws = nv.workspace(dev)
+    out = {}
+    hbm = peaks["hbm_gbs"]
+
+    a, b = wl.tiny_pair()
+    a, b = a.to(dev), b.to(dev)
+    qa, qb = nv.empty(256, 256, device=dev), nv.empty(256, 256, device=dev)
+    y = torch.empty(256, 256, dtype=torch.float32, device=dev)
+    dq = torch.empty(256, 256, dtype=torch.bfloat16, device=dev)
+    t_q = time_flushed(lambda: nv.quantize(a, out=qa, ws=ws), flush)
+    nv.quantize(b, out=qb, ws=ws)
+    t_dq = time_flushed(lambda: nv.dequantize(qa, out=dq), flush)
+    t_g = time_flushed(lambda: nv.gemm(qa, qb, out=y, ws=ws), flush)
+
+    def tiny_all():
+        nv.quantize(a, out=qa, ws=ws)
+        nv.quantize(b, out=qb, ws=ws)
+        nv.dequantize(qa, out=dq)
+        nv.dequantize(qb, out=dq)
+        nv.gemm(qa, qb, out=y, ws=ws)
+    t_all = time_flushed(tiny_all, flush)
+    out["tiny_256"] = {"quantize_us": t_q * 1e3, "dequantize_us": t_dq * 1e3,
+                       "gemm_us": t_g * 1e3, "round_trip_and_gemm_us": t_all * 1e3,
+                       "note": "latency-bound: 2 quantizations, 2 dequantizations, one GEMM"}
+
+    w = wl.qkv()
+    x, wq = w.a.to(dev), nv.quantize(w.w.to(dev))
+    del w
+    qx = nv.empty(M, D, device=dev)
+    yq = torch.empty(M, QKV, dtype=torch.bfloat16, device=dev)
+    flops = 2 * M * QKV * D
+    qbytes = M * D * Q_BYTES_PER_ELEM + 4
+    t_q = time_flushed(lambda: nv.quantize(x, out=qx, ws=ws), flush)
+    t_g = time_flushed(lambda: nv.gemm(qx, wq, out=yq, ws=ws), flush)
+    t_all = time_flushed(lambda: (nv.quantize(x, out=qx, ws=ws), nv.gemm(qx, wq, out=yq, ws=ws)),
+                         flush)
+    out["qkv_projection"] = {"tflops": flops / (t_all * 1e-3) / 1e12, "us": t_all * 1e3,
+                             "gemm_tflops": flops / (t_g * 1e-3) / 1e12, "gemm_us": t_g * 1e3,
+                             "quantize_gb_s": qbytes / (t_q * 1e-3) / 1e9,
+                             "quantize_frac_hbm": qbytes / (t_q * 1e-3) / 1e9 / hbm,
+                             "quantize_us": t_q * 1e3}
+    del x, wq, qx, yq
+
+    f = wl.ffn()
+    x, wu, wd = f.x.to(dev), nv.quantize(f.w_up.to(dev)), nv.quantize(f.w_down.to(dev))
+    del f
+    qx, qh = nv.empty(M, D, device=dev), nv.empty(M, F, device=dev)
+    h = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+    yd = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+
+    def ffn_chain():
+        nv.quantize(x, out=qx, ws=ws)
+        nv.gemm(qx, wu, out=h, ws=ws, c_amax=amax, act=nv.ACT_GELU_TANH)
+        nv.quantize(h, out=qh, ws=ws, amax_in=amax)
+        nv.gemm(qh, wd, out=yd, ws=ws)
+    flops = 2 * 2 * M * F * D
+    t_all = time_flushed(ffn_chain, flush)
+    rq_bytes = M * F * Q_BYTES_PER_ELEM + 4
+    t_rq = time_flushed(lambda: nv.quantize(h, out=qh, ws=ws), flush)
+    out["ffn_pair"] = {"tflops": flops / (t_all * 1e-3) / 1e12, "us": t_all * 1e3,
+                       "requant_gb_s": rq_bytes / (t_rq * 1e-3) / 1e9,
+                       "requant_frac_hbm": rq_bytes / (t_rq * 1e-3) / 1e9 / hbm,
+                       "requant_us_with_amax_pass": t_rq * 1e3}
+    del x, wu, wd, qx, qh, h, yd
+
+    k, v = wl.kv_window()
+    k, v = k.to(dev), v.to(dev)
+    cache = nv.KVCache(WINDOW, TPF, wl.HEADS, wl.HEAD_DIM, device=dev)
+    kw, vw = torch.empty_like(k), torch.empty_like(v)
+    slots = list(range(WINDOW))
+
+    def kv_quant():
+        cache.quant_chunk(k[:8 * TPF], v[:8 * TPF], slots[:8], ws=ws)
+        cache.quant_chunk(k[8 * TPF:], v[8 * TPF:], slots[8:], ws=ws)
+
+    elems = 2 * WINDOW * KV_ELEMS_FRAME
+    qb_ = elems * Q_BYTES_PER_ELEM + 2 * 2 * 4
+    db_ = elems * Q_BYTES_PER_ELEM
+    t_q = time_flushed(kv_quant, flush)
+    t_d = time_flushed(lambda: cache.dequant_window(slots, kw, vw), flush)
+    t_all = time_flushed(lambda: (kv_quant(), cache.dequant_window(slots, kw, vw)), flush)
+    out["kv_codec"] = {"gb_s": (qb_ + db_) / (t_all * 1e-3) / 1e9,
+                       "frac_hbm": (qb_ + db_) / (t_all * 1e-3) / 1e9 / hbm, "us": t_all * 1e3,
+                       "quant_gb_s": qb_ / (t_q * 1e-3) / 1e9,
+                       "quant_frac_hbm": qb_ / (t_q * 1e-3) / 1e9 / hbm,
+                       "dequant_gb_s": db_ / (t_d * 1e-3) / 1e9,
+                       "dequant_frac_hbm": db_ / (t_d * 1e-3) / 1e9 / hbm,
+                       "note": "quant: 2 chunks (8 + 4 frames) x K,V with amax passes"}
+    out["timing"] = "each workload alone, L2 flushed before every call, median of 20"
+    return out
+
+
+def library_fp4_gemm(dev) -> dict:
+    """Context only: cuBLASLt's NVFP4 GEMM (through torch) on the step's four
+    GEMM shapes, fed the same NVFP4 operands as nvfp4_gemm (tensor-core scale
+    layout), timed back to back like the step's launches (30 calls, same
+    operands).  Never on the path; a yardstick for the FP4 tensor peak."""
+    import torch.nn.functional as Fn
+    res = {}
+    g = torch.Generator(device=dev).manual_seed(1)
+    for name, (m, n, k) in GEMM_SHAPES.items():
+        try:
+            qa = nv.quantize(torch.randn(m, k, device=dev, generator=g).to(torch.bfloat16))
+            qw = nv.quantize((torch.randn(n, k, device=dev, generator=g) * 0.02)
+                             .to(torch.bfloat16))
+            out = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+            ws = nv.workspace(dev)
+            a4 = qa.codes.view(torch.float4_e2m1fn_x2)
+            w4 = qw.codes.view(torch.float4_e2m1fn_x2)
+            sa, sw = qa.sf.view(torch.float8_e4m3fn), qw.sf.view(torch.float8_e4m3fn)
+
+            def lib():
+                return Fn.scaled_mm(a4, w4.t(), sa, Fn.ScalingType.BlockWise1x16, sw,
+                                    Fn.ScalingType.BlockWise1x16,
+                                    swizzle_a=Fn.SwizzleType.SWIZZLE_32_4_4,
+                                    swizzle_b=Fn.SwizzleType.SWIZZLE_32_4_4,
+                                    output_dtype=torch.bfloat16)
+
+            def ours():
+                nv.gemm(qa, qw, out=out, ws=ws)
+            r = {}
+            for tag, fn in (("cublaslt", lib), ("nvfp4_gemm", ours)):
+                for _ in range(3):
+                    fn()
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(30):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) / 30 * 1e3
+                r[tag] = {"us": us, "tflops": 2 * m * n * k / us / 1e6}
+            res[name] = r
+        except Exception as e:  # a library without the NVFP4 path: report, do not fail
+            res[name] = {"unavailable": str(e)[:200]}
+    return res
+
+
+def run_case(args) -> int:
+    """One kernel on one step-shaped case, `reps` times, for profilers:
+    ncu -k <kernel> -s <launches to skip> -c <n> python bench.py --case <name>."""
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(7)
+    ws = nv.workspace(dev)
+    case, reps = args.case, args.reps
+    gemm_cases = {"gemm_qkv": ("qkv", nv.ACT_NONE), "gemm_out": ("out", nv.ACT_NONE),
+                  "gemm_up": ("up", nv.ACT_GELU_TANH), "gemm_down": ("down", nv.ACT_NONE)}
+    if case in gemm_cases:
+        shape, act = gemm_cases[case]
+        m, n, k = GEMM_SHAPES[shape]
+        qa = nv.quantize(torch.randn(m, k, device=dev, generator=g).to(torch.bfloat16))
+        qw = nv.quantize((torch.randn(n, k, device=dev, generator=g) * 0.02).to(torch.bfloat16))
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+        run = lambda: nv.gemm(qa, qw, out=out, ws=ws, act=act)  # noqa: E731
+    elif case in ("quant_act", "quant_ffn"):
+        cols = D if case == "quant_act" else F
+        x = torch.randn(M, cols, device=dev, generator=g).to(torch.bfloat16)
+        q = nv.empty(M, cols, device=dev)
+        st = nv.quantize(x).s_t.clone()
+        # the encode pass alone, as in the step (tensor scale handed in)
+        run = lambda: nv.quantize(x, out=q, ws=ws, s_t=st)  # noqa: E731
+    elif case in ("kv_quant", "kv_quant_fos", "kv_dequant", "attention"):
+        rule = nv.SCALE_FOUR_OVER_SIX if case == "kv_quant_fos" else nv.SCALE_ONTO_6
+        cache = nv.KVCache(POOL, TPF, wl.HEADS, wl.HEAD_DIM, device=dev, scale_rule=rule)
+        qkv = torch.randn(M, QKV, device=dev, generator=g).to(torch.bfloat16)
+        for s0 in (0, 3, 6, 9):
+            cache.quant_chunk(qkv[:, D:2 * D], qkv[:, 2 * D:], [s0, s0 + 1, s0 + 2], ws=ws)
+        window = [0, 1, 2, 6, 7, 8, 9, 10, 11, 12, 13, 14]
+        kw = torch.empty(WINDOW * TPF, wl.HEADS, wl.HEAD_DIM, dtype=torch.bfloat16, device=dev)
+        vw = torch.empty_like(kw)
+        o = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+        if case in ("kv_quant", "kv_quant_fos"):
+            run = lambda: cache.quant_chunk(qkv[:, D:2 * D], qkv[:, 2 * D:],  # noqa: E731
+                                            [12, 13, 14], ws=ws)
+        elif case == "kv_dequant":
+            cache.quant_chunk(qkv[:, D:2 * D], qkv[:, 2 * D:], [12, 13, 14], ws=ws)
+            run = lambda: cache.dequant_window(window, kw, vw)  # noqa: E731
+        else:
+            cache.quant_chunk(qkv[:, D:2 * D], qkv[:, 2 * D:], [12, 13, 14], ws=ws)
+            run = lambda: cache.window_attention(qkv[:, :D], window, out=o)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown case {case!r}")
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        run()
+    torch.cuda.synchronize()
+    status = nv.device_status(ws)
+    if status:
+        raise SystemExit(f"device status {status}")
+    print(f"{case}: {reps} reps ok")
+    return 0
+
+
 def run_ours(args):
     world = env_int("WORLD_SIZE", 1)
     rank = env_int("RANK", 0)
@@ -432,7 +573,7 @@ def run_ours(args):
         if dist is not None:
             dist.barrier()
 
-    step = Step(args.layers, dev)
+    step = DiTStep(args.layers, dev)
     stream = torch.cuda.Stream(device=dev)
     # eager warm-up (first calls set kernel attributes), then capture one step
     with torch.cuda.stream(stream):
@@ -523,7 +664,18 @@ def run_ours(args):
     attn_ms = time_window_attention(step, dev)
 
     peaks, peak_src = measured_peaks()
-    fp4_peak = 4.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # FP4 has no measured peak: 4 x the measured bf16 GEMM (the dense FP4:BF16
+    # ratio).  The burst figure applies when the timed region ran at (near) the
+    # maximum SM clock with no power cap, the sustained one (taken under the
+    # power cap at a lower clock) otherwise.
+    burst = 4.0 * peaks["bf16_tflops"]
+    sustained = 4.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    at_max = bool(clock_info and clock_info.get("sm_mhz") and clock_info.get("sm_max_mhz")
+                  and clock_info["sm_mhz"] >= 0.95 * clock_info["sm_max_mhz"]
+                  and "sw_power_cap" not in clock_info.get("reasons", []))
+    if clock_info is None:
+        at_max = True
+    fp4_peak = burst if at_max else sustained
     gemm_tflops = flops_step / (gemm_ms * 1e-3) / 1e12
     codec = {}
     for k in ("quant_act", "requant_ffn", "kv_quant", "kv_dequant"):
@@ -534,12 +686,18 @@ def run_ours(args):
     kv_ms = kernel_ms["kv_quant"] + kernel_ms["kv_dequant"]
     traffic = gemm_traffic_per_launch()
 
+    configs = None if args.no_configs else time_configs(dev, peaks)
+    library = None if args.no_configs else library_fp4_gemm(dev)
+
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             r = CpuSample(rows=args.cpu_rows).run()
             cpu = {"value": r["tflops"], "unit": "TFLOP/s", "cores": r["cores"],
                    "kind": "oracle", "sample": r["sample"], "kv_codec_gbs": r["kv_gbs"]}
+            r1 = CpuSample(rows=args.cpu_rows_1core, threads=1).run()
+            cpu["one_core"] = {"value": r1["tflops"], "unit": "TFLOP/s", "cores": r1["cores"],
+                               "sample": r1["sample"], "kv_codec_gbs": r1["kv_gbs"]}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -549,10 +707,18 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel",
                          "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": gemm_tflops / fp4_peak,
-                         "peak_source": f"{peak_src}: 4 x bf16_tflops_sustained "
-                                        f"({peaks.get('bf16_tflops_sustained')}), nominal "
-                                        "FP4:BF16 dense ratio 4",
-                         "traffic": traffic},
+                         "peak_source": (f"{peak_src}: 4 x bf16_tflops "
+                                         f"({'burst' if at_max else 'sustained'}: "
+                                         f"{peaks['bf16_tflops'] if at_max else peaks.get('bf16_tflops_sustained')}"
+                                         f"), nominal FP4:BF16 dense ratio 4; chosen from the "
+                                         f"clock record (median {clock_info and clock_info.get('sm_mhz')}"
+                                         f" MHz of max {clock_info and clock_info.get('sm_max_mhz')})"),
+                         "frac_vs_sustained": gemm_tflops / sustained,
+                         "frac_vs_nominal_9pf": gemm_tflops / 9000.0,
+                         "traffic": traffic,
+                         "traffic_note": "ncu dram__bytes_read + dram__bytes_write per launch "
+                                         "(writes still in L2 when a launch ends are not "
+                                         "counted)"},
             "kv_codec": {"gb_s": kv_bytes / (kv_ms * 1e-3) / 1e9,
                          "frac_hbm": kv_bytes / (kv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "hbm_peak_gbs": peaks["hbm_gbs"]},
@@ -571,6 +737,10 @@ def run_ours(args):
                      "launches_per_step": gemm_launches,
                      "by_shape_ms": {k: v for k, v in kernel_ms.items() if k.startswith("gemm")}},
             "kernel_ms_per_step": kernel_ms,
+            "kernel_ms_note": "CUDA events between every launch of a second graph of the step "
+                              "(removes the PDL overlap); quant_act includes the amax passes",
+            "configs": configs,
+            "library_fp4_gemm_context": library,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * D * 2,
                     "d2h_bytes_per_step": M * D * 2, "ms_per_step": ms_e2e / args.steps},
@@ -594,8 +764,19 @@ def main():
     ap.add_argument("--layers", type=int, default=wl.LAYERS)
     ap.add_argument("--ref-rows", type=int, default=16, help="rows per reference-arm step")
     ap.add_argument("--cpu-rows", type=int, default=128, help="rows of the cpu_baseline sample")
+    ap.add_argument("--cpu-rows-1core", type=int, default=16,
+                    help="rows of the one-core cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the single-call workload timings and the library comparison")
+    ap.add_argument("--case", default=None,
+                    help="profiling: run one kernel on a step-shaped case --reps times "
+                         "(gemm_qkv gemm_out gemm_up gemm_down quant_act quant_ffn kv_quant "
+                         "kv_quant_fos kv_dequant attention)")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -334,6 +334,10 @@ NVFP4_API int64_t nvfp4_sink_plan_frame_of_slot(const nvfp4_sink_plan* plan, int
  * NVFP4_ERR_UNSUPPORTED_SHAPE, as in nvfp4_quantize.
  *   - The first call on each device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after a
+ *     cudaDeviceReset (or anything else that destroys the device's primary
+ *     context) it is stale, so do not call this entry point on that device
+ *     again in the same process.
  *   - Each call first clears the scratch words on `stream`.  All calls on a
  *     device share the one array, so calls that may overlap on the GPU (other
  *     streams, other threads) race and must be serialized by the caller.

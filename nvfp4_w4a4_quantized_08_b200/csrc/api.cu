@@ -19,20 +19,23 @@ struct DeviceInfo {
 };
 
 // Compute capability and SM count of the current device, cached per device.
+// Host threads may call in concurrently: an entry is published through its
+// atomic word (0 = not yet queried, else 1 + sm_count, negated when the
+// device is not sm_100), so a reader sees either nothing or a whole entry.
 DeviceInfo current_device() {
-  static DeviceInfo cache[64];
-  static bool filled[64] = {};
+  static std::atomic<int> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return {false, 0};
-  if (!filled[dev]) {
+  int word = cache[dev].load(std::memory_order_acquire);
+  if (word == 0) {
     int major = 0, minor = 0, sms = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = {major == 10 && minor == 0, sms};
-    filled[dev] = true;
+    word = (major == 10 && minor == 0) ? 1 + sms : -(1 + sms);
+    cache[dev].store(word, std::memory_order_release);
   }
-  return cache[dev];
+  return {word > 0, (word > 0 ? word : -word) - 1};
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

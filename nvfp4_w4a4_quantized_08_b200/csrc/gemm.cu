@@ -33,6 +33,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -690,15 +691,17 @@ template <bool kGelu>
 static cudaError_t launch_form(const CUtensorMap& map_a, const CUtensorMap& map_w,
                                const CUtensorMap& map_c, const gemm::Params& p, int grid,
                                cudaStream_t st) {
-  static int configured_device = -1;
+  // the shared-memory opt-in is per device; host threads may race here, and
+  // setting the attribute twice is harmless, so each device keeps one flag
+  static std::atomic<bool> configured[64];
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel<kGelu>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          gemm::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured_device = dev;
+    configured[dev].store(true, std::memory_order_release);
   }
   return launch_pdl(gemm::nvfp4_gemm_kernel<kGelu>, dim3(grid), dim3(gemm::kThreads),
                     size_t(gemm::kSmemBytes), st, map_a, map_w, map_c, p);

@@ -27,7 +27,12 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array for the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached.  The cache never expires:
+// the address belongs to the device's primary context, so a cudaDeviceReset
+// leaves it stale (the header tells callers not to use this entry point on a
+// device after resetting it).  The status word at kWsStatus is written by a
+// kernel that meets an out-of-domain tensor scale and never read or cleared:
+// nothing here reports it.
 cudaError_t scratch_address(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
   if (!g_scratch_ptr[dev]) {

@@ -1,7 +1,9 @@
 """GPU: the tensor amax handed from a GEMM epilogue to the next quantization.
 
-The NVFP4 recipe's tensor scale is s_t = amax(x) / (6 * 448) ("Pretraining
-Large Language Models with NVFP4", section 4: two-level scaling).  When x is
+The recipe's tensor scale is s_t = amax(x) / (6 * 448): the FP32 tensor-level
+scale of the two-level NVFP4 scaling (tailorednewshub.com LongLive-2.0 article,
+section "Entrenamiento NVFP4"), with the amax mapped onto the largest E2M1
+value times the largest E4M3 value.  When x is
 the output of an nvfp4_gemm, the GEMM can accumulate max|x| over the values it
 stores (c_amax) and nvfp4_quantize can take that word (amax_in) instead of
 running its own amax pass.  These tests check that the hand-off changes no
