@@ -8,28 +8,47 @@
 // accumulated in FP32 in tensor memory; the tensor-scale product s_tA * s_tW
 // is applied once in the epilogue.
 //
-// Structure: one persistent CTA per SM walks 128 x 256 output tiles.
+// What sets the speed.  The tensor core finishes a 128 x 256 x 64 FP4 step in
+// about 128 clocks, so it needs each step's operand bytes (and their scales)
+// delivered into the SM that fast; operand delivery from L2, not the tensor
+// pipe, is the limit.  Two things follow:
+//   * bytes per MAC: in the pair form a cluster of two CTAs on two SMs computes
+//     a 256 x 256 tile with one cta_group::2 MMA per K step.  Each CTA stages
+//     its own 128 rows of A and its own half of the tile's 256 W rows, and the
+//     pair's tensor cores read both halves of W, so a CTA loads 32 KB of codes
+//     per 128 x 256 x 256 of work instead of 48 KB (one CTA alone, 128 x 256);
+//   * bytes in flight: a stage comes back a load latency after it is
+//     requested, so the ring must hold enough stages to cover that latency;
+//     the pair form's smaller stages leave room for five.
+// The single form (one CTA, 128 x 256 tiles, cta_group::1) serves M <= 128.
+//
+// Warp roles (every CTA of either form):
 //   warp 0      TMA producer: 2-D tensor copies of the A and W code tiles
 //               (128-byte K slabs, 128-byte swizzle) and 1-D bulk copies of the
-//               matching 512-byte scale tiles into a 3-stage shared-memory ring.
-//   warp 1      tensor-core issuer: one MMA per K = 64 step once that step's
-//               scales are in tensor memory; it also owns the tensor-memory
-//               allocation.
-//   warps 2..5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
-//               s_tA * s_tW, round to bf16 / fp32, stage in swizzled shared
-//               memory, TMA tensor store (rows past M are clipped by the store).
-//   warps 6..9  scale writers: per stage, each writes the scale words its lane
-//               quadrant reads into that stage's tensor-memory scale set
-//               (tcgen05.st), off the tensor pipe, which would otherwise run
-//               the scale copies (tcgen05.cp) and the MMAs one after the other,
-//               and hands the set to the issuer through a named barrier.
+//               matching 512-byte scale tiles into the shared-memory ring.
+//   warp 1      tensor-memory owner; lane 0 of the issuing CTA (the pair's
+//               leader, or the single CTA) issues one MMA per K = 64 step and
+//               one commit per stage.
+//   warps 2..9  epilogue: two warps per tensor-memory lane quadrant, each
+//               reading half of the accumulator's 256 columns: tcgen05.ld,
+//               scale by s_tA * s_tW, activation, round to bf16 / fp32, stage
+//               in swizzled shared memory, TMA tensor store (rows past M are
+//               clipped by the store).
+//   warps 10..13 scale writers: per stage, each writes the scale words its
+//               lane quadrant reads into that stage's tensor-memory scale set
+//               (tcgen05.st), off the tensor pipe.
+// Hand-offs are mbarriers: full[s] (this CTA's TMA bytes landed -> writers),
+// sf_ready[s] (the writers of every CTA of the tile -> issuer), empty[s] (the
+// stage's MMAs completed -> every producer; a multicast commit in the pair),
+// acc_full (the tile's MMAs completed -> every epilogue) and acc_empty (every
+// epilogue warp read the accumulator out -> issuer).
 // Tensor memory: the 128 x 256 FP32 accumulator in columns [0,256) and one
-// 48-column scale set per shared-memory stage after it.  The epilogue reads the
-// whole accumulator into registers and releases it before its stores, so the
-// tensor pipe idles only for that read-out between tiles.
+// 48-column scale set per shared-memory stage after it.
 // Every spin-wait is bounded (wait_limit_ns).  A wait that runs out records
-// NVFP4_ERR_TIMEOUT, raises a CTA-wide abort flag, and the CTA drains its own
-// copies, MMAs and stores in flight before freeing tensor memory and returning.
+// NVFP4_ERR_TIMEOUT, raises the CTA's abort flag, and the CTA drains its own
+// copies, MMAs and stores in flight before freeing tensor memory; the CTAs of
+// a pair meet at a cluster barrier before either frees its tensor memory, so
+// neither leaves while the leader's MMAs may still read its operands.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,46 +61,50 @@
 namespace nvfp4 {
 namespace gemm {
 
-constexpr int kBM = 128;          // tile rows (A rows)
-constexpr int kBN = 256;          // tile cols (W rows)
+constexpr int kBM = 128;          // rows of A per CTA (accumulator lanes)
+constexpr int kBN = 256;          // W rows per tile (accumulator columns)
 constexpr int kBKBytes = 128;     // K slab per stage: 128 bytes = 256 FP4 values
-constexpr int kStages = 3;
 constexpr int kKSteps = 4;        // MMA K = 64 values = 32 bytes
 constexpr int kABytes = kBM * kBKBytes;      // 16 KB
-constexpr int kBBytes = kBN * kBKBytes;      // 32 KB
 constexpr int kSfaBytes = 4 * 512;           // 4 scale tiles of 128 rows x 4 blocks
 constexpr int kSfbBytes = 2 * 4 * 512;       // 2 row tiles of W
-constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr int kWriterWarp0 = 2 + kEpiWarps;  // 10
+constexpr int kThreads = (kWriterWarp0 + 4) * 32;  // 448
 constexpr int kTmemCols = 512;
 constexpr int kSfCol = kBN;                  // scale sets after the accumulator
-constexpr int kSfSets = kStages;             // one scale set per shared-memory stage
 constexpr int kSfStepCols = 12;              // per K step: SFA at +0, SFB at +4 and +8
 constexpr int kSfSetCols = kKSteps * kSfStepCols;
 constexpr int kStageBufBytes = 32 * 128;     // epilogue staging: 32 rows x 128 bytes
-constexpr int kEpiWarps = 4;
 
-// shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kStages * kABytes;
-constexpr int kOffSfa = kOffB + kStages * kBBytes;
-constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
-constexpr int kOffStage = kOffSfb + kStages * kSfbBytes;            // 1024-aligned
-constexpr int kOffBar = kOffStage + kEpiWarps * 2 * kStageBufBytes;
-// full[], empty[], acc_full, (unused), acc_release, drain
-constexpr int kNumBars = 2 * kStages + 4;
-constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
-constexpr int kOffAbort = kOffTmemPtr + 4;
-constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
-static_assert(kOffStage % 1024 == 0, "staging buffers need 1024-byte alignment");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kSfCol + kSfSets * kSfSetCols <= kTmemCols, "tensor memory budget");
-static_assert(kBN <= kSfCol, "the accumulator overlaps the scale slots");
-
-// Instruction descriptor, block-scaled kinds: E2M1 A and B (format 1 at bits
-// 7-9 and 10-12), K-major both, N >> 3 at bits 17-22, E4M3 scales (bit 23 = 0),
-// M >> 4 at bits 24-28, scale-factor ids 0.
-constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
-                            (uint32_t(kBM >> 4) << 24);
+// Per-form sizes: kPair = 1 (single CTA) or 2 (CTA pair).
+template <int kPair>
+struct Cfg {
+  static constexpr int kStages = kPair == 2 ? 5 : 3;
+  static constexpr int kBRows = kBN / kPair;             // W rows staged per CTA
+  static constexpr int kBBytes = kBRows * kBKBytes;      // 16 KB / 32 KB
+  static constexpr int kTileM = kBM * kPair;             // output rows per tile
+  // shared memory map (offsets from a 1024-byte aligned base)
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kABytes;
+  static constexpr int kOffSfa = kOffB + kStages * kBBytes;
+  static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
+  static constexpr int kOffStage = kOffSfb + kStages * kSfbBytes;  // 1024-aligned
+  static constexpr int kOffBar = kOffStage + kEpiWarps * kStageBufBytes;
+  // full[], empty[], sf_ready[], acc_full, acc_empty, drain
+  static constexpr int kNumBars = 3 * kStages + 3;
+  static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmemPtr + 4;
+  static constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
+  // Instruction descriptor, block-scaled kinds: E2M1 A and B (format 1 at bits
+  // 7-9 and 10-12), K-major both, N >> 3 at bits 17-22, E4M3 scales (bit 23 =
+  // 0), M >> 4 at bits 24-28 (M of the whole pair for cta_group::2), scale ids 0.
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
+                                     (uint32_t(kTileM >> 4) << 24);
+  static_assert(kOffStage % 1024 == 0, "staging buffers need 1024-byte alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kSfCol + kStages * kSfSetCols <= kTmemCols, "tensor memory budget");
+};
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -113,13 +136,43 @@ __device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity,
   return ok != 0;
 }
 
-__device__ __forceinline__ void bar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of this CTA's shared variable `addr` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (default semantics:
+// release at CTA scope; a cluster-scope release costs the thread about 1000
+// clocks a call).  What an arrival publishes needs no wider release: scale
+// words are in tensor memory once tcgen05.wait::st returns, and an epilogue
+// warp's tensor-memory reads are complete once tcgen05.wait::ld returns; both
+// are ordered for the issuer's tensor-core work by the tcgen05 fences around
+// the hand-off.
+__device__ __forceinline__ void bar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void bar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Every thread of every CTA of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void bar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x,
@@ -147,10 +200,61 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Arrive on `bar` once the tcgen05 operations issued so far complete: in this
+// CTA (single form), or at the same address in both CTAs of the pair.
+template <int kPair>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-      : "memory");
+  if constexpr (kPair == 1) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+  } else {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"(uint16_t(3))
+        : "memory");
+  }
+}
+
+// Arrive on this CTA's `bar` only (the drain barrier).
+template <int kPair>
+__device__ __forceinline__ void tc_commit_local(uint32_t bar) {
+  if constexpr (kPair == 1) {
+    tc_commit<1>(bar);
+  } else {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+  }
+}
+
+template <int kPair>
+__device__ __forceinline__ void tmem_alloc(uint32_t dst) {
+  if constexpr (kPair == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+}
+
+template <int kPair>
+__device__ __forceinline__ void tmem_dealloc(uint32_t tmem) {
+  if constexpr (kPair == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  } else {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -160,16 +264,27 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+template <int kPair>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
-      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
+  if constexpr (kPair == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+  }
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -184,16 +299,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Named barriers 1..kSfSets hand a stage's scales from the 4 writer warps
-// (arrive) to the issuer warp (sync).
-constexpr int kNamedBarThreads = 5 * 32;
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t threads) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // One 32-bit column of this warp's 32 tensor-memory lanes from a register.
@@ -297,9 +402,9 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, 
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// Wait until at most one committed store group still reads shared memory.
-__device__ __forceinline__ void bulk_wait_read_le1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+// Wait until no committed store group still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -312,16 +417,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 }
 
 // One 128-byte segment of each of this warp's 32 output rows (32 words a
-// lane) through the warp's staging buffer (two alternating 4 KB buffers,
-// 128-byte swizzle) and a TMA tensor store at column x, row y.
-__device__ __forceinline__ void store_row_chunk(const uint32_t (&w)[32], uint32_t stage0,
-                                                uint32_t& nstore, int lane, const CUtensorMap* map,
-                                                int32_t x, int32_t y) {
-  const uint32_t sb = stage0 + (nstore & 1) * kStageBufBytes;
-  // the store issued two chunks ago must have finished reading this buffer
-  if (lane == 0) bulk_wait_read_le1();
+// lane) through the warp's 4 KB staging buffer (128-byte swizzle) and a TMA
+// tensor store at column x, row y.
+__device__ __forceinline__ void store_row_chunk(const uint32_t (&w)[32], uint32_t buf, int lane,
+                                                const CUtensorMap* map, int32_t x, int32_t y) {
+  // the previous store from this buffer must have finished reading it
+  if (lane == 0) bulk_wait_read_all();
   __syncwarp();
-  const uint32_t row = sb + uint32_t(lane) * 128;
+  const uint32_t row = buf + uint32_t(lane) * 128;
   const uint32_t sw = uint32_t(lane) & 7;  // 128-byte swizzle: 16-byte unit ^ (row % 8)
 #pragma unroll
   for (uint32_t u = 0; u < 8; ++u)
@@ -329,10 +432,9 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&w)[32], uint32_
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(map, x, y, sb);
+    tma_store_2d(map, x, y, buf);
     bulk_commit();
   }
-  ++nstore;
 }
 
 struct Params {
@@ -343,7 +445,8 @@ struct Params {
   uint32_t M, N;
   uint32_t ktiles;   // K / 64
   uint32_t kslabs;   // ceil(K / 256)
-  uint32_t tiles_m, tiles_n;
+  uint32_t tiles_m, tiles_n;  // output tiles: tiles_m of 128 * kPair rows, tiles_n of 256 cols
+  uint32_t sf_row_tiles;      // 128-row blocks of A that exist (ceil(M / 128))
   uint32_t* status;
   uint32_t* c_amax;  // float bits of max|C| (atomicMax), or null
   uint32_t amax_tiles;  // N tiles per c_amax word (0: one word)
@@ -351,47 +454,52 @@ struct Params {
   int32_t c_dtype;
 };
 
-template <bool kGelu>
+template <int kPair, bool kGelu>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                       const __grid_constant__ CUtensorMap map_w,
                       const __grid_constant__ CUtensorMap map_c, const Params p) {
+  using C = Cfg<kPair>;
+  constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + kOffBar;                 // + 8 s
+  const uint32_t bar_full = sbase + C::kOffBar;              // + 8 s
   const uint32_t bar_empty = bar_full + 8 * kStages;         // + 8 s
-  const uint32_t bar_acc_full = bar_empty + 8 * kStages;     // + 8 b
-  const uint32_t bar_acc_release = bar_acc_full + 16;
-  const uint32_t bar_drain = bar_acc_release + 8;
-  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  const uint32_t bar_sf = bar_empty + 8 * kStages;           // + 8 s (issuing CTA)
+  const uint32_t bar_acc_full = bar_sf + 8 * kStages;
+  const uint32_t bar_acc_empty = bar_acc_full + 8;           // issuing CTA
+  const uint32_t bar_drain = bar_acc_empty + 8;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::kOffTmemPtr);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // rank in the pair (0 = leader, the CTA that issues the MMAs)
+  const uint32_t rank = kPair == 2 ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       bar_init(bar_full + 8 * s, 1);
       bar_init(bar_empty + 8 * s, 1);
+      bar_init(bar_sf + 8 * s, 4 * kPair);  // every scale-writer warp of the tile
     }
     bar_init(bar_acc_full, 1);
-    bar_init(bar_acc_release, kEpiWarps);
+    bar_init(bar_acc_empty, kEpiWarps * kPair);
     bar_init(bar_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_ptr)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 1) tmem_alloc<kPair>(smem_u32(tmem_ptr));
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair == 2) {
+    cluster_sync();  // the peer's barriers are initialised before any remote arrival
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
   // on-chip setup done; from here on global memory is read and written
@@ -400,6 +508,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const Waiter waiter{p.wait_limit_ns, abort_flag, p.status};
   const uint32_t num_tiles = p.tiles_m * p.tiles_n;
+  // tiles are walked per CTA (single) or per pair, both CTAs of a pair in step
+  const uint32_t t0 = blockIdx.x / kPair, t_step = gridDim.x / kPair;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -408,21 +518,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(&map_w) : "memory");
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
-      for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (uint32_t t = t0; t < num_tiles && ok; t += t_step) {
         const uint32_t tm = t % p.tiles_m, tn = t / p.tiles_m;
+        // this CTA's 128-row block of A; past the last one (a pair's follower
+        // when the row blocks run out) the code loads read zeros and no scales
+        // are loaded
+        const uint32_t rt = tm * kPair + rank;
+        const bool a_live = rt < p.sf_row_tiles;
         for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
           if (!waiter.wait(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
           const uint32_t fb = bar_full + 8 * stage;
-          bar_arrive_expect_tx(fb, kABytes + kBBytes + 3 * 512 * nk);
-          tma_load_2d(sbase + kOffA + stage * kABytes, &map_a, int32_t(kb * kBKBytes),
-                      int32_t(tm * kBM), fb);
-          tma_load_2d(sbase + kOffB + stage * kBBytes, &map_w, int32_t(kb * kBKBytes),
-                      int32_t(tn * kBN), fb);
-          bulk_load(sbase + kOffSfa + stage * kSfaBytes,
-                    p.a_sf + (size_t(tm) * p.ktiles + kb * kKSteps) * 512, 512 * nk, fb);
+          bar_arrive_expect_tx(fb, kABytes + C::kBBytes + (a_live ? 3u : 2u) * 512u * nk);
+          tma_load_2d(sbase + C::kOffA + stage * kABytes, &map_a, int32_t(kb * kBKBytes),
+                      int32_t(rt * kBM), fb);
+          tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &map_w, int32_t(kb * kBKBytes),
+                      int32_t(tn * kBN + rank * C::kBRows), fb);
+          if (a_live)
+            bulk_load(sbase + C::kOffSfa + stage * kSfaBytes,
+                      p.a_sf + (size_t(rt) * p.ktiles + kb * kKSteps) * 512, 512 * nk, fb);
+          // the scales of all 256 W rows of the tile, in either form
           for (uint32_t h = 0; h < 2; ++h)
-            bulk_load(sbase + kOffSfb + stage * kSfbBytes + h * 2048,
+            bulk_load(sbase + C::kOffSfb + stage * kSfbBytes + h * 2048,
                       p.w_sf + (size_t(2 * tn + h) * p.ktiles + kb * kKSteps) * 512, 512 * nk,
                       fb);
           ++issued;
@@ -435,108 +552,121 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar_full + 8 * s, (last / kStages) & 1, p.status);
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Lane 0 issues; the whole warp takes part in the named-barrier handoff
-    // from the scale writers (bar.sync counts whole warps).  The MMAs of a
-    // stage hold the issuing thread until the tensor pipe accepts them, so
-    // everything between two stages is kept short: one handoff, one commit.
-    // Every writer arrives once per stage, aborting or not, so the bar.sync
-    // below always completes.
-    uint32_t stage = 0, phase = 0, local = 0;
-    bool ok = true;
-    for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
-      // the previous tile's epilogue must have read the accumulator out
-      if (local > 0) {
-        bool released = true;
-        if (lane == 0) released = waiter.wait(bar_acc_release, (local - 1) & 1);
-        if (!__shfl_sync(0xFFFFFFFFu, released, 0)) break;
-      }
-      for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
-        // the writers have seen this stage land (they waited on its full
-        // barrier) and put its scales in set `stage`; the named barrier orders
-        // this thread after their observation
-        named_bar_sync(1 + stage, kNamedBarThreads);
-        if (*abort_flag) { ok = false; break; }
-        if (lane == 0) {
+    // One thread of the issuing CTA.  Per stage: wait until the writers of
+    // every CTA of the tile have put the stage's scales in tensor memory (they
+    // did so after seeing the stage's operands land), issue the stage's MMAs,
+    // commit them to the stage's empty barrier (both CTAs' in a pair).  Per
+    // tile: wait until every epilogue warp read the previous accumulator out,
+    // and commit the tile's MMAs to acc_full.
+    if (leader && lane == 0) {
+      uint32_t stage = 0, phase = 0, local = 0;
+      bool ok = true;
+      for (uint32_t t = t0; t < num_tiles && ok; t += t_step, ++local) {
+        if (local > 0 && !waiter.wait(bar_acc_empty, (local - 1) & 1)) break;
+        tc_fence_after();
+        for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
+          if (!waiter.wait(bar_sf + 8 * stage, phase)) { ok = false; break; }
           tc_fence_after();
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
-          const uint64_t a_d = desc_sw128(sbase + kOffA + stage * kABytes);
-          const uint64_t b_d = desc_sw128(sbase + kOffB + stage * kBBytes);
+          const uint64_t a_d = desc_sw128(sbase + C::kOffA + stage * kABytes);
+          const uint64_t b_d = desc_sw128(sbase + C::kOffB + stage * C::kBBytes);
           const uint32_t sf = tmem + kSfCol + kSfSetCols * stage;
           for (uint32_t j = 0; j < nk; ++j)  // K step j: +32 bytes = +2 in the address field
-            tc_mma(tmem, a_d + 2 * j, b_d + 2 * j, kIdesc, sf + kSfStepCols * j,
-                   sf + kSfStepCols * j + 4, (kb | j) != 0);
-          // frees the shared-memory stage and its scale set once these MMAs complete
-          tc_commit(bar_empty + 8 * stage);
+            tc_mma<kPair>(tmem, a_d + 2 * j, b_d + 2 * j, C::kIdesc, sf + kSfStepCols * j,
+                          sf + kSfStepCols * j + 4, (kb | j) != 0);
+          // frees the shared-memory stage and its scale set (of both CTAs of a
+          // pair) once these MMAs complete
+          tc_commit<kPair>(bar_empty + 8 * stage);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
-        __syncwarp();
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (!ok) break;
+        tc_commit<kPair>(bar_acc_full);
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(bar_acc_full);
-      __syncwarp();
-    }
-    // drain: every tcgen05 operation this warp issued has completed
-    if (lane == 0) {
-      tc_commit(bar_drain);
+      // drain: every tcgen05 operation this thread issued has completed
+      tc_commit_local<kPair>(bar_drain);
       drain_wait(bar_drain, 0, p.status);
     }
     __syncwarp();
-  } else if (warp >= 2 + kEpiWarps) {
+  } else if (warp >= kWriterWarp0) {
     // ------------------------------------------------------------ scale writers
     // Each warp owns one tensor-memory lane quadrant q; lane quadrant q of the
-    // tensor core computes output rows 32q..32q+31.  A staged scale tile is 32
-    // chunks of 16 bytes, chunk l holding the four E4M3 scales of rows l,
-    // l+32, l+64, l+96 of a 128-row operand tile.  Per K step the MMA reads
+    // tensor core computes output rows 32q..32q+31 of this CTA's 128.  A staged
+    // scale tile is 32 chunks of 16 bytes, chunk l holding the four E4M3 scales
+    // of rows l, l+32, l+64, l+96 of a 128-row operand tile.  Per K step the
+    // MMA reads
     //   A scales of row 32q + l: lane 32q + l, column sfa + q (its own rows);
     //   W scales of row n (any of the 256, every quadrant needs them all):
     //     lane 32q + n % 32, column sfb + n / 32.
-    // So warp q writes word q of A chunk `lane` into one column and both W
-    // chunks `lane` whole (4 columns each) into its lanes, a stage at a time,
-    // into the stage's scale set, then hands it to the issuer through named
-    // barrier 1 + stage.  A set is free when its stage is full again: the
-    // producer refilled the stage after the MMAs that read the set completed.
+    // In a pair each CTA's tensor memory holds the same layout for its own 128
+    // rows of A and all 256 W rows of the tile.  So warp q writes word q of A
+    // chunk `lane` into one column and both W chunks `lane` whole (4 columns
+    // each) into its lanes, a stage at a time, into the stage's scale set, then
+    // arrives on the issuing CTA's sf_ready barrier of the stage.  A set is free
+    // when its stage is full again: the producer refilled the stage after the
+    // MMAs that read the set completed.
     const uint32_t q = uint32_t(warp & 3);
     const uint32_t lane_bits = (q * 32) << 16;
+    const uint32_t sf_bar0 = kPair == 2 && !leader ? map_to_rank(bar_sf, 0) : bar_sf;
     uint32_t stage = 0, phase = 0;
     bool ok = true;
-    for (uint32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+    for (uint32_t t = t0; t < num_tiles && ok; t += t_step) {
       for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
         ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_full + 8 * stage, phase));
-        if (ok) {
-          tc_fence_after();
-          const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
-          const uint32_t sfa_s = sbase + kOffSfa + stage * kSfaBytes + 16 * uint32_t(lane) + 4 * q;
-          const uint32_t sfb_s = sbase + kOffSfb + stage * kSfbBytes + 16 * uint32_t(lane);
-          const uint32_t col = tmem + lane_bits + kSfCol + kSfSetCols * stage;
-          for (uint32_t j = 0; j < nk; ++j) {
-            tmem_st1(col + kSfStepCols * j + q, ld_shared_u32(sfa_s + 512 * j));
-            tmem_st4(col + kSfStepCols * j + 4, ld_shared_v4(sfb_s + 512 * j));
-            tmem_st4(col + kSfStepCols * j + 8, ld_shared_v4(sfb_s + 2048 + 512 * j));
-          }
-          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-          tc_fence_before();
-        }
-        // arrive even when aborting: the issuer is (or will be) waiting here
-        named_bar_arrive(1 + stage, kNamedBarThreads);
         if (!ok) break;
+        tc_fence_after();
+        const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
+        const uint32_t sfa_s = sbase + C::kOffSfa + stage * kSfaBytes + 16 * uint32_t(lane) + 4 * q;
+        const uint32_t sfb_s = sbase + C::kOffSfb + stage * kSfbBytes + 16 * uint32_t(lane);
+        const uint32_t col = tmem + lane_bits + kSfCol + kSfSetCols * stage;
+        for (uint32_t j = 0; j < nk; ++j) {
+          tmem_st1(col + kSfStepCols * j + q, ld_shared_u32(sfa_s + 512 * j));
+          tmem_st4(col + kSfStepCols * j + 4, ld_shared_v4(sfb_s + 512 * j));
+          tmem_st4(col + kSfStepCols * j + 8, ld_shared_v4(sfb_s + 2048 + 512 * j));
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (kPair == 2 && !leader) {
+            bar_arrive_remote(sf_bar0 + 8 * stage);
+          } else {
+            bar_arrive(sf_bar0 + 8 * stage);
+          }
+        }
         if (++stage == kStages) { stage = 0; phase ^= 1; }
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // The accumulator is read out whole into registers (bf16: 128 packed words
-    // a thread; fp32: two halves of 128 words), scaled by s_tA * s_tW and
-    // released to the MMA issuer before the stores, so the next tile's MMAs
-    // wait only for the reads.  The activation (kGelu) takes the bf16 products
-    // after the release (fp32 output: the fp32 products, as they are read).
-    const uint32_t ew = uint32_t(warp - 2);            // staging buffers of this warp
+    // Warp w (2..9) reads lane quadrant w % 4 (its 32 output rows) and columns
+    // [128 h, 128 h + 128), h = (w - 2) / 4, of the accumulator into registers
+    // (bf16: 64 packed words a thread), scales by s_tA * s_tW and releases the
+    // accumulator before its stores, so the next tile's MMAs wait only for the
+    // reads.  For bf16 output the activation (kGelu) takes the bf16 products
+    // after the release; for fp32 output it runs as the values are read.
+    const uint32_t ew = uint32_t(warp - 2);
     const uint32_t quad = uint32_t(warp & 3);          // tensor-memory lane quadrant
+    const uint32_t half = ew >> 2;                     // column half of the tile
     const float alpha = __fmul_rn(*p.a_st, *p.w_st);
     const bool bf16 = p.c_dtype == NVFP4_BF16;
-    const uint32_t stage0 = sbase + kOffStage + ew * 2 * kStageBufBytes;
-    uint32_t local = 0, nstore = 0;
+    const uint32_t buf = sbase + C::kOffStage + ew * kStageBufBytes;
+    const uint32_t acc_empty =
+        kPair == 2 && !leader ? map_to_rank(bar_acc_empty, 0) : bar_acc_empty;
+    auto release = [&]() {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (kPair == 2 && !leader) {
+          bar_arrive_remote(acc_empty);
+        } else {
+          bar_arrive(acc_empty);
+        }
+      }
+    };
+    uint32_t local = 0;
     // running max of |stored value| as magnitude bits (two bf16 halves, or
     // fp32) for c_amax word `word`; flushed when the tiles move to another word
     uint32_t vmax = 0, word = 0;
@@ -548,24 +678,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && wmax != 0) atomicMax(p.c_amax + word, wmax);
       vmax = 0;
     };
-    for (uint32_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+    for (uint32_t t = t0; t < num_tiles; t += t_step, ++local) {
       const uint32_t tm = t % p.tiles_m, tn = t / p.tiles_m;
       if (want_max && p.amax_tiles > 0 && tn / p.amax_tiles != word) {
         flush_max();
         word = tn / p.amax_tiles;
       }
-      // accumulator lanes past the last row of C hold zeros; leave them out anyway
-      const bool row_live = want_max && tm * kBM + quad * 32 + uint32_t(lane) < p.M;
-      const int32_t y = int32_t(tm * kBM + quad * 32);
+      const uint32_t row0 = (tm * kPair + rank) * kBM + quad * 32;  // this warp's first row
+      // accumulator lanes past the last row of C hold no output; leave them out
+      const bool row_live = want_max && row0 + uint32_t(lane) < p.M;
+      const bool store = row0 < p.M;  // warp-uniform: some of the 32 rows exist
+      const int32_t y = int32_t(row0);
+      const int32_t x0 = int32_t(tn * kBN + half * 128);
       // warp-uniform outcome: tcgen05.ld below is .sync.aligned
       const bool ok = waiter.wait(bar_acc_full, local & 1);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + ((quad * 32) << 16);
+      const uint32_t taddr = tmem + ((quad * 32) << 16) + half * 128;
       if (bf16) {
-        uint32_t pk[128];
+        uint32_t pk[64];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
           tmem_ld32(taddr + 32 * c, r);
 #pragma unroll
@@ -573,49 +706,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[16 * c + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
                                        __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) bar_arrive(bar_acc_release);
+        release();
         // the activation runs on the bf16 products once the accumulator is
         // released, overlapping the next tile's MMAs: a bf16 linear layer
         // followed by its activation
         if (kGelu) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e) pk[e] = gelu_bf16x2(pk[e]);
+          for (int e = 0; e < 64; ++e) pk[e] = gelu_bf16x2(pk[e]);
         }
         if (row_live) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e) vmax = __vmaxu2(vmax, pk[e] & 0x7FFF7FFFu);
+          for (int e = 0; e < 64; ++e) vmax = __vmaxu2(vmax, pk[e] & 0x7FFF7FFFu);
         }
+        if (store) {
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          store_row_chunk(*reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * ch]), stage0, nstore,
-                          lane, &map_c, int32_t(tn * kBN + 64 * ch), y);
+          for (int ch = 0; ch < 2; ++ch)
+            store_row_chunk(*reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * ch]), buf, lane,
+                            &map_c, x0 + 64 * ch, y);
+        }
       } else {
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t v[128];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr + 32 * c, v);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(taddr + 128 * half + 32 * c, r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              v[32 * c + e] = __float_as_uint(epi<kGelu>(__uint_as_float(r[e]), alpha));
-          }
-          if (half == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) bar_arrive(bar_acc_release);
-          }
+          for (int e = 0; e < 32; ++e)
+            v[e] = __float_as_uint(epi<kGelu>(__uint_as_float(v[e]), alpha));
+          if (c == 3) release();
           if (row_live) {
 #pragma unroll
-            for (int e = 0; e < 128; ++e) vmax = max(vmax, v[e] & 0x7FFFFFFFu);
+            for (int e = 0; e < 32; ++e) vmax = max(vmax, v[e] & 0x7FFFFFFFu);
           }
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
-            store_row_chunk(*reinterpret_cast<const uint32_t(*)[32]>(&v[32 * ch]), stage0,
-                            nstore, lane, &map_c, int32_t(tn * kBN + 128 * half + 32 * ch), y);
+          if (store) store_row_chunk(v, buf, lane, &map_c, x0 + 32 * c, y);
         }
       }
     }
@@ -626,13 +748,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols)
-                 : "memory");
+  if constexpr (kPair == 2) {
+    // neither CTA of the pair frees tensor memory or leaves while the leader's
+    // MMAs (drained above) or the follower's arrivals may still touch the other
+    cluster_sync();
+  } else {
+    __syncthreads();
   }
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc<kPair>(tmem);
 }
 
 }  // namespace gemm
@@ -687,32 +811,67 @@ static bool make_out_map(CUtensorMap* map, void* base, int32_t dtype, uint64_t r
   return r == CUDA_SUCCESS;
 }
 
-template <bool kGelu>
+// The pair form whenever A has more than one 128-row block: it computes the
+// same tiles with half the W bytes per CTA and half the MMA instructions.
+static bool use_pair(int64_t M) { return M > gemm::kBM; }
+
+template <int kPair, bool kGelu>
 static cudaError_t launch_form(const CUtensorMap& map_a, const CUtensorMap& map_w,
-                               const CUtensorMap& map_c, const gemm::Params& p, int grid,
+                               const CUtensorMap& map_c, const gemm::Params& p, int sm_count,
                                cudaStream_t st) {
+  using C = gemm::Cfg<kPair>;
   // the shared-memory opt-in is per device; host threads may race here, and
   // setting the attribute twice is harmless, so each device keeps one flag
-  static std::atomic<bool> configured[64];
+  // (configured[dev] holds 1 + the number of CTAs -- single -- or pairs that
+  // can be resident at once)
+  static std::atomic<int> configured[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev].load(std::memory_order_acquire)) {
-    cudaError_t e = cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel<kGelu>,
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(gemm::kThreads);
+  cfg.dynamicSmemBytes = size_t(C::kSmemBytes);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = kPair;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kPair == 2 ? 2 : 1;
+  int slots = configured[dev].load(std::memory_order_acquire) - 1;
+  if (slots < 0) {
+    cudaError_t e = cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel<kPair, kGelu>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         gemm::kSmemBytes);
+                                         C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured[dev].store(true, std::memory_order_release);
+    slots = sm_count / kPair;
+    if (kPair == 2) {
+      // pairs must sit on two SMs of one GPC: ask how many fit at once
+      int n = 0;
+      cfg.gridDim = dim3(2 * slots);
+      if (cudaOccupancyMaxActiveClusters(&n, gemm::nvfp4_gemm_kernel<kPair, kGelu>, &cfg) ==
+              cudaSuccess &&
+          n > 0 && n < slots)
+        slots = n;
+    }
+    configured[dev].store(slots + 1, std::memory_order_release);
   }
-  return launch_pdl(gemm::nvfp4_gemm_kernel<kGelu>, dim3(grid), dim3(gemm::kThreads),
-                    size_t(gemm::kSmemBytes), st, map_a, map_w, map_c, p);
+  const uint32_t tiles = p.tiles_m * p.tiles_n;
+  cfg.gridDim = dim3(kPair * int(tiles < uint32_t(slots) ? tiles : uint32_t(slots)));
+  return cudaLaunchKernelEx(&cfg, gemm::nvfp4_gemm_kernel<kPair, kGelu>, map_a, map_w, map_c, p);
 }
 
 cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
+  const bool pair = use_pair(g.M);
+  const uint32_t w_box_rows = pair ? uint32_t(gemm::Cfg<2>::kBRows) : uint32_t(gemm::kBN);
   CUtensorMap map_a, map_w, map_c;
   if (!make_code_map(&map_a, g.a_codes, uint64_t(g.K / 2), uint64_t(g.M), gemm::kBM) ||
-      !make_code_map(&map_w, g.w_codes, uint64_t(g.K / 2), uint64_t(g.N), gemm::kBN) ||
+      !make_code_map(&map_w, g.w_codes, uint64_t(g.K / 2), uint64_t(g.N), w_box_rows) ||
       !make_out_map(&map_c, g.c, g.c_dtype, uint64_t(g.M), uint64_t(g.N), uint64_t(g.ldc)))
     return cudaErrorInvalidValue;
+  const int64_t tile_m = pair ? 2 * gemm::kBM : gemm::kBM;
   gemm::Params p;
   p.a_sf = g.a_sf;
   p.w_sf = g.w_sf;
@@ -722,17 +881,20 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.N = uint32_t(g.N);
   p.ktiles = uint32_t(g.K / 64);
   p.kslabs = uint32_t((g.K + 255) / 256);
-  p.tiles_m = uint32_t((g.M + gemm::kBM - 1) / gemm::kBM);
+  p.tiles_m = uint32_t((g.M + tile_m - 1) / tile_m);
   p.tiles_n = uint32_t(g.N / gemm::kBN);
+  p.sf_row_tiles = uint32_t((g.M + gemm::kBM - 1) / gemm::kBM);
   p.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(g.ws) + kWsStatus);
   p.c_amax = reinterpret_cast<uint32_t*>(g.c_amax);
   p.amax_tiles = uint32_t(g.c_amax_cols / gemm::kBN);
   p.wait_limit_ns = g.wait_limit_ns;
   p.c_dtype = g.c_dtype;
-  const uint32_t tiles = p.tiles_m * p.tiles_n;
-  const int grid = int(tiles < uint32_t(g.sm_count) ? tiles : uint32_t(g.sm_count));
-  return g.act == NVFP4_ACT_GELU_TANH ? launch_form<true>(map_a, map_w, map_c, p, grid, st)
-                                      : launch_form<false>(map_a, map_w, map_c, p, grid, st);
+  const bool gelu = g.act == NVFP4_ACT_GELU_TANH;
+  if (pair)
+    return gelu ? launch_form<2, true>(map_a, map_w, map_c, p, g.sm_count, st)
+                : launch_form<2, false>(map_a, map_w, map_c, p, g.sm_count, st);
+  return gelu ? launch_form<1, true>(map_a, map_w, map_c, p, g.sm_count, st)
+              : launch_form<1, false>(map_a, map_w, map_c, p, g.sm_count, st);
 }
 
 }  // namespace nvfp4

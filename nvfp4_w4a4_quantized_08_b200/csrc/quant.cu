@@ -284,21 +284,34 @@ __device__ __forceinline__ void fill_inv_table(float* tab) {
     tab[b] = (b == 0 || b == 0x7F) ? 0.0f : __frcp_rn(e4m3_to_f32(b));
 }
 
-// Thread 0 of every CTA calls this once.  It returns the plane's tensor scale:
-// s_t_in if given, else amax / 2688 with the amax the producer accumulated
-// (amax_in) or the one this call's amax pass left in the workspace.  An amax
-// word is read once per CTA; the CTA then checks in on the plane's counter
-// (release: the read is ordered before the check-in) and the CTA that checks
-// in last (acquire: every other read happened before) zeroes the amax word and
-// the counter for the next call.  Checking in right after the read keeps the
-// wait for the atomic off the CTA's exit.
-__device__ __forceinline__ float take_scale(const float* s_t_in, float* amax_in, uint32_t* ws,
-                                            int plane) {
+// The plane's tensor scale: s_t_in if given, else amax / 2688 with the amax
+// the producer accumulated (amax_in) or the one this call's amax pass left in
+// the workspace.  Every thread reads the word itself, so no thread waits for
+// another before it starts encoding.
+__device__ __forceinline__ float read_scale(const float* s_t_in, const float* amax_in,
+                                            const uint32_t* ws, int plane) {
   if (s_t_in) return *s_t_in;
+  const uint32_t* const word =
+      amax_in ? reinterpret_cast<const uint32_t*>(amax_in) : ws + kWsAmax0 / 4 + plane;
+  uint32_t bits;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(bits) : "l"(word) : "memory");
+  return __fdiv_rn(__uint_as_float(bits), 2688.0f);
+}
+
+// Every CTA calls this once, after all of its threads have read the amax word
+// (a CTA barrier first).  Thread 0 checks the CTA in on the plane's counter
+// (release: the CTA's reads are ordered before the check-in); the CTA that
+// checks in last (acquire: every other CTA's reads happened before) zeroes the
+// amax word and the counter for the next call.  Nothing to do when the scale
+// was handed in as s_t_in.
+__device__ __forceinline__ void check_in(const float* s_t_in, float* amax_in, uint32_t* ws,
+                                         int plane) {
+  if (s_t_in) return;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
   uint32_t* const word = amax_in ? reinterpret_cast<uint32_t*>(amax_in) : ws + kWsAmax0 / 4 + plane;
   uint32_t* const counter = ws + kWsCount0 / 4 + plane;
-  uint32_t bits, done;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(bits) : "l"(word) : "memory");
+  uint32_t done;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
                : "=r"(done)
                : "l"(counter)
@@ -307,7 +320,6 @@ __device__ __forceinline__ float take_scale(const float* s_t_in, float* amax_in,
     asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(word) : "memory");
     asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(counter) : "memory");
   }
-  return __fdiv_rn(__uint_as_float(bits), 2688.0f);
 }
 
 // Input blocks a thread keeps in flight while it encodes the ones it holds.
@@ -459,8 +471,8 @@ template <typename InT, bool kContig, int kSfLayout>
 __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args) {
   constexpr int D = Prefetch<InT>::kDepth;
   __shared__ float inv_tab[128];
-  __shared__ float s_t_shared;
   fill_inv_table(inv_tab);
+  __syncthreads();
   pdl_wait();
   pdl_trigger();
   const uint32_t stride = gridDim.x * blockDim.x;
@@ -472,9 +484,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args)
     const uint32_t b = b0 + i * stride;
     load_block<InT>(block_ptr<InT, kContig>(args.in, min(b, blocks - 1)), cur[i]);
   }
-  if (threadIdx.x == 0) s_t_shared = take_scale(args.s_t_in, args.amax_in, args.ws, 0);
-  __syncthreads();
-  const float s_t = s_t_shared;
+  const float s_t = read_scale(args.s_t_in, args.amax_in, args.ws, 0);
   const bool in_domain = tensor_scale_in_domain(s_t);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     *args.s_t_out = s_t;
@@ -527,6 +537,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args)
       args.sf[sf_mma_offset(row, kb, args.ktiles)] = 0;
     }
   }
+  check_in(args.s_t_in, args.amax_in, args.ws, 0);
 }
 
 // ---- KV-cache chunks (K and V planes in one launch, blockIdx.y)
@@ -548,8 +559,8 @@ __global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4
     kv_quant_kernel(KvQuantArgs args) {
   constexpr int D = Prefetch<__nv_bfloat16>::kDepth;
   __shared__ float inv_tab[128];
-  __shared__ float s_t_shared;
   fill_inv_table(inv_tab);
+  __syncthreads();
   pdl_wait();
   pdl_trigger();
   const int plane = blockIdx.y;
@@ -564,10 +575,8 @@ __global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4
     load_block<__nv_bfloat16>(block_ptr<__nv_bfloat16, kContig>(m, min(b, blocks - 1)),
                               cur[i]);
   }
-  if (threadIdx.x == 0)
-    s_t_shared = take_scale(nullptr, plane == 0 ? args.amax_in[0] : args.amax_in[1], args.ws, plane);
-  __syncthreads();
-  const float s_t = s_t_shared;
+  float* const amax_in = plane == 0 ? args.amax_in[0] : args.amax_in[1];
+  const float s_t = read_scale(nullptr, amax_in, args.ws, plane);
   const bool in_domain = tensor_scale_in_domain(s_t);
   if (blockIdx.x == 0 && threadIdx.x < args.n_frames)
     args.st[plane][args.slots[threadIdx.x]] = s_t;
@@ -606,6 +615,7 @@ __global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4
       }
     }
   }
+  check_in(nullptr, amax_in, args.ws, plane);
 }
 
 // ---------------------------------------------------------------- launchers
