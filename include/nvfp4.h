@@ -275,12 +275,17 @@ NVFP4_API nvfp4_status nvfp4_kv_dequant_window(const nvfp4_kv_cache* cache, cons
  *        this reads Q straight out of a fused QKV projection output.
  *   softmax_scale: finite, > 0 (usually 1 / sqrt(head_dim)).
  *   out: device bf16, tq tokens at out_token_stride, same layout as q.
+ *   ws:  device workspace of ws_bytes >= nvfp4_workspace_bytes() (its status
+ *        word records a bounded wait that ran out: NVFP4_ERR_TIMEOUT, read by
+ *        nvfp4_get_device_status; the limit is nvfp4_set_wait_limit_ns's).
  *   head_dim must be 128.
- * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, ARCH, CUDA. */
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, ARCH, CUDA;
+ * TIMEOUT via the status word. */
 NVFP4_API nvfp4_status nvfp4_window_attention(const nvfp4_kv_cache* cache, const int32_t* slot_ids,
                                               int32_t n, const void* q, int64_t q_token_stride,
                                               int64_t tq, float softmax_scale, void* out,
-                                              int64_t out_token_stride, void* stream);
+                                              int64_t out_token_stride, void* ws, size_t ws_bytes,
+                                              void* stream);
 
 /* Slot planning for multi-shot generation (host only: no device work, no
  * stream).  Each chunk of new frames attends to three sets of frames

@@ -108,7 +108,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_sink_plan_frame_of_slot.argtypes = [vp, i32]
         L.nvfp4_window_attention.restype = i32
         L.nvfp4_window_attention.argtypes = [KP, ctypes.POINTER(ctypes.c_int32), i32, vp, i64,
-                                             i64, ctypes.c_float, vp, i64, vp]
+                                             i64, ctypes.c_float, vp, i64, vp, ctypes.c_size_t,
+                                             vp]
         L.nvfp4_get_device_status.restype = i32
         L.nvfp4_get_device_status.argtypes = [vp, vp]
         L.nvfp4_set_wait_limit_ns.restype = None

@@ -137,6 +137,7 @@ nvfp4_status nvfp4_quantize(const void* x, int32_t dtype, int64_t rows, int64_t 
   q.amax_in = amax_in;
   q.ws = ws;
   q.sm_count = dev.sm_count;
+  q.wait_limit_ns = g_wait_limit_ns.load();
   return cuda_status(launch_quantize(q, static_cast<cudaStream_t>(stream)));
 }
 
@@ -249,6 +250,7 @@ nvfp4_status nvfp4_kv_quant_chunk(const nvfp4_kv_cache* cache, const void* k, co
   q.scale_rule = cache->scale_rule;
   q.ws = ws;
   q.sm_count = dev.sm_count;
+  q.wait_limit_ns = g_wait_limit_ns.load();
   return cuda_status(launch_kv_quant(q, static_cast<cudaStream_t>(stream)));
 }
 
@@ -286,7 +288,7 @@ nvfp4_status nvfp4_kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t*
 nvfp4_status nvfp4_window_attention(const nvfp4_kv_cache* cache, const int32_t* slot_ids,
                                     int32_t n, const void* q, int64_t q_token_stride, int64_t tq,
                                     float softmax_scale, void* out, int64_t out_token_stride,
-                                    void* stream) {
+                                    void* ws, size_t ws_bytes, void* stream) {
   nvfp4_status st = check_cache(cache);
   if (st != NVFP4_OK) return st;
   if (!slot_ids || !q || !out || n < 1 || n > NVFP4_KV_MAX_WINDOW_SLOTS)
@@ -302,6 +304,8 @@ nvfp4_status nvfp4_window_attention(const nvfp4_kv_cache* cache, const int32_t* 
   if (!aligned(q, 16) || !aligned(out, 16) || q_token_stride % 8 != 0 ||
       out_token_stride % 8 != 0)
     return NVFP4_ERR_MISALIGNED;
+  if (!ws || ws_bytes < kWsBytes) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;
   const DeviceInfo dev = current_device();
   if (!dev.ok) return NVFP4_ERR_ARCH;
   LaunchAttn d;
@@ -321,6 +325,8 @@ nvfp4_status nvfp4_window_attention(const nvfp4_kv_cache* cache, const int32_t* 
   d.out_stride = out_token_stride;
   d.tq = tq;
   d.scale_log2 = float(double(softmax_scale) * 1.4426950408889634);
+  d.ws = ws;
+  d.wait_limit_ns = g_wait_limit_ns.load();
   return cuda_status(launch_window_attention(d, static_cast<cudaStream_t>(stream)));
 }
 

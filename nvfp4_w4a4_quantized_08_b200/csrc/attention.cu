@@ -1,4 +1,5 @@
-// attention.cu -- windowed attention that reads the NVFP4 KV cache directly.
+// attention.cu -- windowed attention that reads the NVFP4 KV cache directly,
+// on the sm_100a tensor cores.
 //
 // The new chunk's queries attend to the frames of the attention window (the
 // sink frames and the local window: 171host.com LongLive 2.0 teardown, section
@@ -7,32 +8,82 @@
 // for windowed attention).  Instead of rebuilding the whole window as bf16 in
 // HBM and reading it back, each CTA decodes the K and V tiles it is about to
 // use into shared memory (the same bf16_RNE((v * s_b) * s_t) values the window
-// rebuild writes) and consumes them at once.
+// rebuild writes) and hands them to the tensor core.
 //
 //   out[t][h] = sum_j softmax_j(scale * q[t][h] . k[j][h]) v[j][h]
 //
 // over the window's tokens j in slot-list order; no mask inside the window
 // (chunk-wise attention: the chunk sees itself and the cached frames whole).
 //
-// Structure: one CTA per (64 queries, head), 4 warps of 16 query rows each.
-// Per 64-token KV tile: all threads decode K into Ks[token][dim] and V
-// transposed into Vt[dim][token] (bf16, padded rows); each warp computes its
-// 16 x 64 scores with mma.sync m16n8k16 (bf16 in, fp32 accumulate), updates the
-// running row max and sum (online softmax in base 2), rounds the probabilities
-// to bf16 and accumulates P V with mma.sync into a 16 x 128 fp32 accumulator.
+// Structure: one CTA per (128 queries, head), 13 warps.
+//   warps 0..3  softmax and epilogue: warp w owns tensor-memory lane quadrant
+//               w, i.e. query rows 32w..32w+31, one row per thread.  They load
+//               Q into shared memory once; per KV tile they read the scores
+//               S = Q K^T of their row out of tensor memory, update the running
+//               row maximum and sum (base 2), and write the probabilities
+//               rounded to bf16 back into tensor memory, where the P V product
+//               reads them as its A operand.
+//   warp 4      tensor-memory owner; lane 0 issues the MMAs
+//               (tcgen05.mma kind::f16, bf16 in, fp32 accumulate):
+//               S_j = Q K_j^T into one of three score buffers, then
+//               O += P_{j-1} V_{j-1}, so the tensor core computes the next
+//               tile's scores while the softmax warps work on the current one.
+//   warps 5..12 decoders: per 128-token tile, the 16-element NVFP4 blocks of
+//               K and V of this head -> bf16 (byte-permute table per block),
+//               K as [token][dim] and V transposed as [dim][token], both in
+//               the tensor core's 128-byte-swizzled K-major layout, into a
+//               two-stage ring.
+// Tensor memory (512 columns): O in [0,128), three score buffers at 128, 256
+// and 384; tile j's scores (then its probabilities) use buffer j % 3, and the
+// issuer writes a buffer again only after the P V product that read it has
+// completed (p_free), which with three buffers it almost never waits for.
+// The running maximum is raised lazily: while a row's new scores stay within
+// 2^8 of the maximum in use, the probabilities are taken against the old one
+// (they stay <= 2^8); only a larger step rescales the row's O and sum, after
+// the previous P V product has completed.  Every wait is bounded: one that
+// runs out records NVFP4_ERR_TIMEOUT in the workspace status word, and the CTA
+// drains its MMAs, frees tensor memory and returns.
 #include "common.cuh"
 #include "decode.cuh"
 #include "kernels.h"
 
-namespace nvfp4 {
+#include <atomic>
 
-constexpr int kAttD = 128;                 // head_dim
-constexpr int kAttBQ = 64;                 // query rows per CTA
-constexpr int kAttBK = 64;                 // KV tokens per tile
-constexpr int kAttThreads = 128;
-constexpr int kLdK = kAttD + 8;            // Ks row: 136 bf16 (272 B, 68 words)
-constexpr int kLdV = kAttBK + 8;           // Vt row: 72 bf16 (144 B, 36 words)
-constexpr int kDimBlocks = kAttD / 16;     // 16-element blocks per token and head
+namespace nvfp4 {
+namespace attn {
+
+constexpr int kD = 128;                   // head_dim
+constexpr int kBQ = 128;                  // queries per CTA (tensor-memory lanes)
+constexpr int kBK = 128;                  // keys per tile
+constexpr int kDimBlocks = kD / 16;       // 16-element blocks per token and head
+constexpr int kSoftWarps = 4;             // warps 0..3
+constexpr int kMmaWarp = 4;
+constexpr int kDecWarp0 = 5;
+constexpr int kDecWarps = 8;
+constexpr int kThreads = (kDecWarp0 + kDecWarps) * 32;  // 416
+constexpr int kStages = 2;
+constexpr int kChunkBytes = 128 * 128;    // 128 rows x 64 bf16 (one K chunk of an operand)
+constexpr int kOpBytes = 2 * kChunkBytes;  // 128 rows x 128 bf16
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kOpBytes;                // + stage * kOpBytes
+constexpr int kOffV = kOffK + kStages * kOpBytes;      // transposed V, + stage * kOpBytes
+constexpr int kOffBar = kOffV + kStages * kOpBytes;
+// q_ready, kv_full[2], kv_empty[2], s_full[3], p_ready[3], p_free[3], pv_done, o_full, drain
+constexpr int kSBufs = 3;
+constexpr int kNumBars = 1 + 2 * kStages + 3 * kSBufs + 3;
+constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+constexpr int kOffAbort = kOffTmemPtr + 4;
+constexpr int kSmemBytes = kOffAbort + 4 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kOCol = 0;
+constexpr uint32_t kSCol0 = 128;          // score buffer b at kSCol0 + 128 b
+// Instruction descriptor, kind::f16: fp32 D (bit 4), bf16 A and B (bits 7 and
+// 10), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBK >> 3) << 17) |
+                            (uint32_t(kBQ >> 4) << 24);
+constexpr float kLazyLog2 = 8.0f;          // largest probability kept before a rescale: 2^8
 
 struct AttnArgs {
   const uint16_t* q;   // bf16 [tq][q_stride], head h at h * 128
@@ -44,201 +95,457 @@ struct AttnArgs {
   uint32_t tq, heads, tpf, n_kv;  // n_kv = window slots * tpf
   FastDiv tpf_div;
   float scale_log2;               // softmax scale * log2(e)
+  uint32_t* status;
+  uint64_t wait_limit_ns;
   int32_t slots[NVFP4_KV_MAX_WINDOW_SLOTS];
 };
 
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(20000)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart, descriptor version 1.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// D (+)= A B^T, A and B in shared memory.
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(acc)
+      : "memory");
+}
+// D (+)= A B^T, A in tensor memory.
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(kIdesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ uint32_t lds32(const uint16_t* p) {
-  return *reinterpret_cast<const uint32_t*>(p);
+// Byte offset of 16-byte unit u (0..15: elements 8u..8u+7) of row r in a
+// 128-row operand tile of 128 bf16 per row, in the tensor core's K-major,
+// 128-byte-swizzled layout (two 64-element chunks of 16 KB).
+__device__ __forceinline__ uint32_t op_offset(uint32_t r, uint32_t u) {
+  return (u >> 3) * kChunkBytes + (r >> 3) * 1024 + (r & 7) * 128 + (((u & 7) ^ (r & 7)) << 4);
 }
 
-__global__ void __launch_bounds__(kAttThreads) window_attention_kernel(const AttnArgs a) {
-  __shared__ __align__(16) uint16_t Ks[kAttBK * kLdK];
-  __shared__ __align__(16) uint16_t Vt[kAttD * kLdV];
-  pdl_wait();
-  pdl_trigger();
-  const uint32_t h = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;  // mma fragment row group / column pair
-  const uint32_t row_a = blockIdx.x * kAttBQ + warp * 16 + g, row_b = row_a + 8;
-
-  // Q fragments of this warp's 16 rows, 8 K steps of 16 dims (rows past tq: 0)
-  uint32_t qa[8][4];
-  {
-    const uint16_t* qra = a.q + int64_t(row_a) * a.q_stride + h * kAttD + 2 * t;
-    const uint16_t* qrb = a.q + int64_t(row_b) * a.q_stride + h * kAttD + 2 * t;
-    const bool va = row_a < a.tq, vb = row_b < a.tq;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      qa[ks][0] = va ? __ldg(reinterpret_cast<const uint32_t*>(qra + 16 * ks)) : 0u;
-      qa[ks][1] = vb ? __ldg(reinterpret_cast<const uint32_t*>(qrb + 16 * ks)) : 0u;
-      qa[ks][2] = va ? __ldg(reinterpret_cast<const uint32_t*>(qra + 16 * ks + 8)) : 0u;
-      qa[ks][3] = vb ? __ldg(reinterpret_cast<const uint32_t*>(qrb + 16 * ks + 8)) : 0u;
+struct Waiter {
+  uint64_t limit_ns;
+  volatile int* abort;
+  uint32_t* status;
+  // Wait for phase `parity` of `bar`; false if the CTA aborted or the wait ran out.
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
+    if (bar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+      if (*abort) return false;
+      if (bar_try_wait(bar, parity)) return true;
+      if (globaltimer() - t0 > limit_ns) {
+        record_status(status, NVFP4_ERR_TIMEOUT);
+        *abort = 1;
+        return false;
+      }
     }
   }
-  float o[16][4];
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
+};
 
-  const uint32_t n_tiles = (a.n_kv + kAttBK - 1) / kAttBK;
-  for (uint32_t kt = 0; kt < n_tiles; ++kt) {
-    __syncthreads();  // every warp is done with the previous tile
-    // ---- decode the K and V blocks of tokens [64 kt, 64 kt + 64) of head h:
-    // 2 planes x 64 tokens x 8 blocks, 8 per thread, every pass's loads issued
-    // before any block is decoded.  K passes (it < 4): token threadIdx / 8 +
-    // 16 it, dim block threadIdx % 8 (a warp's 16-byte row stores spread over
-    // all banks).  V passes: token threadIdx % 64, dim block 2 (it - 4) +
-    // threadIdx / 64, so that a warp's transposed 16-bit stores hit 16
-    // consecutive words of one Vt row (dim-block-major lanes would put all 8
-    // blocks' rows, 16 x 36 words apart, in one bank).
+// Decoded bf16 of one 16-element block of K or V: token w of the window
+// (position w / tpf in the slot list), dim block db of head h; zeros past the
+// window's end.
+__device__ __forceinline__ void load_block(const AttnArgs& a, int plane, uint32_t w, uint32_t h,
+                                           uint32_t db, uint2& c, uint32_t& sb, float& st) {
+  const uint32_t ww = min(w, a.n_kv - 1);
+  const uint32_t pos = fast_div(a.tpf_div, ww);
+  const uint32_t local = ww - pos * a.tpf;
+  const size_t s = size_t(a.slots[pos]);
+  const size_t blk = ((s * a.tpf + local) * a.heads + h) * kDimBlocks + db;
+  c = __ldg(reinterpret_cast<const uint2*>(a.codes[plane]) + blk);
+  sb = __ldg(a.sf[plane] + blk);
+  st = __ldg(a.st[plane] + s);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_q = sbase + kOffBar;
+  const uint32_t bar_kv_full = bar_q + 8;                      // + 8 stage
+  const uint32_t bar_kv_empty = bar_kv_full + 8 * kStages;     // + 8 stage
+  const uint32_t bar_s_full = bar_kv_empty + 8 * kStages;      // + 8 buffer
+  const uint32_t bar_p_ready = bar_s_full + 8 * kSBufs;        // + 8 buffer
+  const uint32_t bar_p_free = bar_p_ready + 8 * kSBufs;        // + 8 buffer
+  const uint32_t bar_pv_done = bar_p_free + 8 * kSBufs;
+  const uint32_t bar_o_full = bar_pv_done + 8;
+  const uint32_t bar_drain = bar_o_full + 8;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t h = blockIdx.y;
+  const uint32_t q0 = blockIdx.x * kBQ;
+  const uint32_t n_tiles = (a.n_kv + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    bar_init(bar_q, kSoftWarps);
+    for (int s = 0; s < kStages; ++s) {
+      bar_init(bar_kv_full + 8 * s, kDecWarps);
+      bar_init(bar_kv_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < kSBufs; ++b) {
+      bar_init(bar_s_full + 8 * b, 1);
+      bar_init(bar_p_ready + 8 * b, kSoftWarps);
+      bar_init(bar_p_free + 8 * b, 1);
+    }
+    bar_init(bar_pv_done, 1);
+    bar_init(bar_o_full, 1);
+    bar_init(bar_drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_ptr)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  pdl_wait();
+  pdl_trigger();
+  const Waiter waiter{a.wait_limit_ns, abort_flag, a.status};
+
+  if (warp < kSoftWarps) {
+    // ------------------------------------------------------------ softmax
+    const uint32_t row = uint32_t(warp) * 32 + uint32_t(lane);   // query row of this thread
+    const uint32_t lane_bits = (uint32_t(warp) * 32) << 16;
+    // Q row -> shared memory (rows past tq are zero)
     {
-      auto tok_of = [](int it) {
-        return it < 4 ? int(threadIdx.x) / kDimBlocks + 16 * it : int(threadIdx.x) % kAttBK;
-      };
-      auto db_of = [](int it) {
-        return it < 4 ? int(threadIdx.x) % kDimBlocks : 2 * (it - 4) + int(threadIdx.x) / kAttBK;
-      };
-      uint2 c[8];
-      uint32_t sb[8];
-      float stv[8];
+      const bool live = q0 + row < a.tq;
+      const uint4* src =
+          reinterpret_cast<const uint4*>(a.q + int64_t(q0 + (live ? row : 0)) * a.q_stride + h * kD);
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int plane = it / 4;
-        const int tok = tok_of(it), db = db_of(it);
-        const uint32_t j = min(kt * kAttBK + tok, a.n_kv - 1);  // past the end: reload, zeroed below
-        const uint32_t pos = fast_div(a.tpf_div, j);  // position in the slot list
-        const uint32_t local = j - pos * a.tpf;
-        const size_t s = size_t(a.slots[pos]);
-        const size_t blk = ((s * a.tpf + local) * a.heads + h) * kDimBlocks + db;
-        c[it] = __ldg(reinterpret_cast<const uint2*>(a.codes[plane]) + blk);
-        sb[it] = __ldg(a.sf[plane] + blk);
-        stv[it] = __ldg(a.st[plane] + s);
+      for (uint32_t u = 0; u < 16; ++u) {
+        const uint4 v = live ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+        st_shared_v4(sbase + kOffQ + op_offset(row, u), v);
       }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) bar_arrive(bar_q);
+    }
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool ok = true;
+    for (uint32_t j = 0; j < n_tiles && ok; ++j) {
+      const uint32_t b = j % kSBufs;
+      ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_s_full + 8 * b, (j / kSBufs) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_bits + kSCol0 + 128 * b;
+      const uint32_t n_valid = min(uint32_t(kBK), a.n_kv - j * kBK);
+      // pass 1: the tile's row maximum (scaled, base 2) over the live keys
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (uint32_t c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(s_addr + 32 * c, r);
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int tok = tok_of(it), db = db_of(it);
-        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-        if (kt * kAttBK + tok < a.n_kv) {
-          const BlockLut l = make_lut(sb[it], stv[it]);
-          lo = decode8(l, c[it].x);
-          hi = decode8(l, c[it].y);
+        for (uint32_t e = 0; e < 32; ++e)
+          if (32 * c + e < n_valid) mx = fmaxf(mx, __fmul_rn(__uint_as_float(r[e]), a.scale_log2));
+      }
+      // lazy maximum: keep the one in use while the tile stays within 2^8 of it
+      float factor = 1.0f;
+      if (mx > m_run + kLazyLog2) {
+        factor = exp2f(m_run - mx);   // 0 on the first tile
+        m_run = mx;
+        l_run = l_run * factor;
+      }
+      // pass 2: probabilities, their sum, bf16 into the score buffer's first
+      // 64 columns (chunk c's 16 words go over columns already read)
+      float sum = 0.0f;
+#pragma unroll 1
+      for (uint32_t c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(s_addr + 32 * c, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (uint32_t e = 0; e < 16; ++e) {
+          const uint32_t k0 = 32 * c + 2 * e;
+          const float p0 = k0 < n_valid
+                               ? exp2f(__fmul_rn(__uint_as_float(r[2 * e]), a.scale_log2) - m_run)
+                               : 0.0f;
+          const float p1 = k0 + 1 < n_valid
+                               ? exp2f(__fmul_rn(__uint_as_float(r[2 * e + 1]), a.scale_log2) - m_run)
+                               : 0.0f;
+          sum += p0 + p1;
+          pk[e] = bf16x2_rn(p0, p1);
         }
-        if (it < 4) {
-          uint4* dst = reinterpret_cast<uint4*>(Ks + tok * kLdK + 16 * db);
-          dst[0] = lo;
-          dst[1] = hi;
-        } else {
-          const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-          uint16_t* col = Vt + (16 * db) * kLdV + tok;
+        tmem_st16(s_addr + 16 * c, pk);
+      }
+      l_run += sum;
+      // a raised maximum rescales this row's O, once the previous P V is done
+      if (__any_sync(0xFFFFFFFFu, factor != 1.0f) && j > 0) {
+        ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_pv_done, (j - 1) & 1));
+        if (ok) {
+          tc_fence_after();
+#pragma unroll 1
+          for (uint32_t c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_bits + kOCol + 32 * c, r);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            col[(2 * e) * kLdV] = uint16_t(w[e] & 0xFFFFu);
-            col[(2 * e + 1) * kLdV] = uint16_t(w[e] >> 16);
+            for (uint32_t e = 0; e < 32; ++e)
+              r[e] = __float_as_uint(__fmul_rn(__uint_as_float(r[e]), factor));
+            tmem_st32(tmem + lane_bits + kOCol + 32 * c, r);
+          }
+        }
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(bar_p_ready + 8 * b);
+    }
+    // ---- epilogue: O / l -> bf16 (rows past tq are not stored)
+    if (ok) ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_o_full, 0));
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.0f / l_run;
+      const bool live = q0 + row < a.tq;
+      uint4* dst = reinterpret_cast<uint4*>(a.out + int64_t(q0 + row) * a.out_stride + h * kD);
+#pragma unroll 1
+      for (uint32_t c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_bits + kOCol + 32 * c, r);
+        if (live) {
+#pragma unroll
+          for (uint32_t e = 0; e < 4; ++e) {
+            uint4 v;
+            v.x = bf16x2_rn(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv);
+            v.y = bf16x2_rn(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv);
+            v.z = bf16x2_rn(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv);
+            v.w = bf16x2_rn(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv);
+            dst[4 * c + e] = v;
           }
         }
       }
     }
-    __syncthreads();
-
-    // ---- S = Q K^T for this warp's 16 rows and the tile's 64 tokens
-    float s[8][4];
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = waiter.wait(bar_q, 0);
+      const uint64_t qd = desc_sw128(sbase + kOffQ);
+      // O += P_jj V_jj: P from score buffer jj % 3, V^T from ring stage jj % 2
+      auto issue_pv = [&](uint32_t jj) {
+        const uint32_t bb = jj % kSBufs, st = jj % kStages;
+        if (!waiter.wait(bar_p_ready + 8 * bb, (jj / kSBufs) & 1)) return false;
+        tc_fence_after();
+        const uint64_t vd = desc_sw128(sbase + kOffV + st * kOpBytes);
+        const uint32_t p_addr = tmem + kSCol0 + 128 * bb;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
-      const uint16_t* krow = Ks + (8 * nt + g) * kLdK + 2 * t;
+        for (uint32_t ks = 0; ks < 8; ++ks)  // 16 keys a step: 8 columns of P, 32 bytes of V^T
+          mma_ts(tmem + kOCol, p_addr + 8 * ks,
+                 vd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3), (jj | ks) != 0);
+        tc_commit(bar_kv_empty + 8 * st);
+        tc_commit(bar_p_free + 8 * bb);
+        tc_commit(bar_pv_done);
+        return true;
+      };
+      for (uint32_t j = 0; j < n_tiles && ok; ++j) {
+        const uint32_t st = j % kStages, b = j % kSBufs;
+        if (!waiter.wait(bar_kv_full + 8 * st, (j / kStages) & 1)) { ok = false; break; }
+        // the P V product that last read score buffer b (tile j - 3) is done
+        if (j >= kSBufs && !waiter.wait(bar_p_free + 8 * b, (j / kSBufs - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t kd = desc_sw128(sbase + kOffK + st * kOpBytes);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) mma_bf16(s[nt], qa[ks], lds32(krow + 16 * ks), lds32(krow + 16 * ks + 8));
-    }
-    // ---- online softmax, base 2: tokens past the window get probability 0
-    float mx_a = -INFINITY, mx_b = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const bool live = kt * kAttBK + 8 * nt + 2 * t + e < a.n_kv;
-        s[nt][e] = live ? __fmul_rn(s[nt][e], a.scale_log2) : -INFINITY;
-        s[nt][2 + e] = live ? __fmul_rn(s[nt][2 + e], a.scale_log2) : -INFINITY;
-        mx_a = fmaxf(mx_a, s[nt][e]);
-        mx_b = fmaxf(mx_b, s[nt][2 + e]);
+        for (uint32_t ks = 0; ks < 8; ++ks)  // 16 dims a step: +32 bytes, next chunk after 4
+          mma_ss(tmem + kSCol0 + 128 * b, qd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3),
+                 kd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3), ks != 0);
+        tc_commit(bar_s_full + 8 * b);
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && issue_pv(n_tiles - 1)) tc_commit(bar_o_full);
+      // drain: every tcgen05 operation this thread issued has completed
+      tc_commit(bar_drain);
+      const uint64_t t0 = globaltimer();
+      while (!bar_try_wait(bar_drain, 0)) {
+        if (globaltimer() - t0 > 2000000000ull) {
+          record_status(a.status, NVFP4_ERR_TIMEOUT);
+          break;
+        }
       }
     }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ decoders
+    const uint32_t t = threadIdx.x - kDecWarp0 * 32;   // 0..255
+    bool ok = true;
+    for (uint32_t j = 0; j < n_tiles && ok; ++j) {
+      const uint32_t b = j % kStages;
+      ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_kv_empty + 8 * b, ((j / kStages) & 1) ^ 1));
+      if (!ok) break;
+      const uint32_t w0 = j * kBK;
+      // K: token t / 8 + 32 i, dim block t % 8 (8 lanes read one token's 64 bytes)
+      uint2 kc[4];
+      uint32_t ksb[4];
+      float kst[4];
 #pragma unroll
-    for (int sh = 1; sh <= 2; sh <<= 1) {
-      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xFFFFFFFFu, mx_a, sh));
-      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xFFFFFFFFu, mx_b, sh));
-    }
-    // every tile holds at least one live token, so the new maxima are finite
-    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-    const float corr_a = exp2f(m_a - mn_a), corr_b = exp2f(m_b - mn_b);
-    m_a = mn_a;
-    m_b = mn_b;
-    float sum_a = 0.0f, sum_b = 0.0f;
+      for (uint32_t i = 0; i < 4; ++i)
+        load_block(a, 0, w0 + t / 8 + 32 * i, h, t % 8, kc[i], ksb[i], kst[i]);
+      // V: token pair p = t % 64 (tokens 2p, 2p + 1), dim block t / 64 + 4 i
+      uint2 vc[2][2];
+      uint32_t vsb[2][2];
+      float vst[2][2];
+      const uint32_t p = t % 64;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+      for (uint32_t i = 0; i < 2; ++i)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        s[nt][e] = exp2f(s[nt][e] - mn_a);
-        s[nt][2 + e] = exp2f(s[nt][2 + e] - mn_b);
-        sum_a += s[nt][e];
-        sum_b += s[nt][2 + e];
+        for (uint32_t e = 0; e < 2; ++e)
+          load_block(a, 1, w0 + 2 * p + e, h, t / 64 + 4 * i, vc[i][e], vsb[i][e], vst[i][e]);
+      const uint32_t kbase = sbase + kOffK + b * kOpBytes;
+#pragma unroll
+      for (uint32_t i = 0; i < 4; ++i) {
+        const uint32_t tok = t / 8 + 32 * i, db = t % 8;
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+        if (w0 + tok < a.n_kv) {
+          const BlockLut l = make_lut(ksb[i], kst[i]);
+          lo = decode8(l, kc[i].x);
+          hi = decode8(l, kc[i].y);
+        }
+        st_shared_v4(kbase + op_offset(tok, 2 * db), lo);
+        st_shared_v4(kbase + op_offset(tok, 2 * db + 1), hi);
       }
-    }
-    l_a = l_a * corr_a + sum_a;
-    l_b = l_b * corr_b + sum_b;
+      const uint32_t vbase = sbase + kOffV + b * kOpBytes;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      o[nt][0] *= corr_a;
-      o[nt][1] *= corr_a;
-      o[nt][2] *= corr_b;
-      o[nt][3] *= corr_b;
-    }
-    // ---- O += P V: P (bf16) as the A operand, 4 K steps of 16 tokens
+      for (uint32_t i = 0; i < 2; ++i) {
+        const uint32_t db = t / 64 + 4 * i;
+        uint32_t wv[2][8];
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint32_t pa[4] = {bf16x2_rn(s[2 * ks][0], s[2 * ks][1]),
-                              bf16x2_rn(s[2 * ks][2], s[2 * ks][3]),
-                              bf16x2_rn(s[2 * ks + 1][0], s[2 * ks + 1][1]),
-                              bf16x2_rn(s[2 * ks + 1][2], s[2 * ks + 1][3])};
+        for (uint32_t e = 0; e < 2; ++e) {
+          uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+          if (w0 + 2 * p + e < a.n_kv) {
+            const BlockLut l = make_lut(vsb[i][e], vst[i][e]);
+            lo = decode8(l, vc[i][e].x);
+            hi = decode8(l, vc[i][e].y);
+          }
+          wv[e][0] = lo.x; wv[e][1] = lo.y; wv[e][2] = lo.z; wv[e][3] = lo.w;
+          wv[e][4] = hi.x; wv[e][5] = hi.y; wv[e][6] = hi.z; wv[e][7] = hi.w;
+        }
+        // V^T row d = 16 db + k holds keys 2p, 2p + 1 in one word
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        const uint16_t* vrow = Vt + (8 * nt + g) * kLdV + 16 * ks + 2 * t;
-        mma_bf16(o[nt], pa, lds32(vrow), lds32(vrow + 8));
+        for (uint32_t k = 0; k < 16; ++k) {
+          const uint32_t d = 16 * db + k;
+          const uint32_t word = prmt(wv[0][k >> 1], wv[1][k >> 1], (k & 1) ? 0x7632u : 0x5410u);
+          st_shared_u32(vbase + op_offset(d, p / 4) + (p % 4) * 4, word);
+        }
       }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) bar_arrive(bar_kv_full + 8 * b);
     }
   }
 
-  // ---- normalise and store (rows past tq are not stored)
-#pragma unroll
-  for (int sh = 1; sh <= 2; sh <<= 1) {
-    l_a += __shfl_xor_sync(0xFFFFFFFFu, l_a, sh);
-    l_b += __shfl_xor_sync(0xFFFFFFFFu, l_b, sh);
-  }
-  const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
-  if (row_a < a.tq) {
-    uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + int64_t(row_a) * a.out_stride + h * kAttD);
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-      dst[4 * nt + t] = bf16x2_rn(o[nt][0] * inv_a, o[nt][1] * inv_a);
-  }
-  if (row_b < a.tq) {
-    uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + int64_t(row_b) * a.out_stride + h * kAttD);
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-      dst[4 * nt + t] = bf16x2_rn(o[nt][2] * inv_b, o[nt][3] * inv_b);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
   }
 }
 
+}  // namespace attn
+
 cudaError_t launch_window_attention(const LaunchAttn& d, cudaStream_t st) {
-  AttnArgs a;
+  attn::AttnArgs a;
   a.q = static_cast<const uint16_t*>(d.q);
   a.out = static_cast<uint16_t*>(d.out);
   a.q_stride = d.q_stride;
@@ -255,9 +562,22 @@ cudaError_t launch_window_attention(const LaunchAttn& d, cudaStream_t st) {
   a.n_kv = uint32_t(d.n * d.tpf);
   a.tpf_div = make_fastdiv(uint32_t(d.tpf));
   a.scale_log2 = d.scale_log2;
+  a.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(d.ws) + kWsStatus);
+  a.wait_limit_ns = d.wait_limit_ns;
   for (int i = 0; i < d.n; ++i) a.slots[i] = d.slot_ids[i];
-  const dim3 grid(uint32_t((d.tq + kAttBQ - 1) / kAttBQ), uint32_t(d.heads));
-  return launch_pdl(window_attention_kernel, grid, dim3(kAttThreads), 0, st, a);
+  static std::atomic<bool> configured[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev].load(std::memory_order_acquire)) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        attn::window_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attn::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev].store(true, std::memory_order_release);
+  }
+  const dim3 grid(uint32_t((d.tq + attn::kBQ - 1) / attn::kBQ), uint32_t(d.heads));
+  return launch_pdl(attn::window_attention_kernel, grid, dim3(attn::kThreads),
+                    size_t(attn::kSmemBytes), st, a);
 }
 
 }  // namespace nvfp4

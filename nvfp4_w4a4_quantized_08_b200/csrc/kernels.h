@@ -21,6 +21,7 @@ struct LaunchQuant {
   float* amax_in;  // producer-accumulated amax (consumed and reset), or NULL
   void* ws;
   int sm_count;
+  uint64_t wait_limit_ns;
 };
 cudaError_t launch_quantize(const LaunchQuant& q, cudaStream_t st);
 
@@ -47,6 +48,7 @@ struct LaunchKvQuant {
   int32_t scale_rule;            // nvfp4_scale_rule
   void* ws;
   int sm_count;
+  uint64_t wait_limit_ns;
 };
 cudaError_t launch_kv_quant(const LaunchKvQuant& q, cudaStream_t st);
 
@@ -70,6 +72,8 @@ struct LaunchAttn {
   void* out;                // bf16
   int64_t q_stride, out_stride, tq;
   float scale_log2;         // softmax scale * log2(e)
+  void* ws;                 // workspace (status word)
+  uint64_t wait_limit_ns;
 };
 cudaError_t launch_window_attention(const LaunchAttn& d, cudaStream_t st);
 

@@ -93,5 +93,6 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int32_t dtype, int
   q.amax_in = nullptr;
   q.ws = scratch;
   q.sm_count = sms;
+  q.wait_limit_ns = 2000000000ull;
   return launch_quantize(q, st) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -205,7 +205,8 @@ class KVCache:
 
     def window_attention(self, q: torch.Tensor, slot_ids: Sequence[int],
                          scale: Optional[float] = None,
-                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                         out: Optional[torch.Tensor] = None,
+                         ws: Optional[torch.Tensor] = None) -> torch.Tensor:
         """nvfp4_window_attention: softmax(scale q k^T) v over the listed slots,
         read straight from the NVFP4 pools.  q: bf16 [tq, >= heads*head_dim]
         (row stride a multiple of 8, e.g. the Q third of a QKV output) ->
@@ -224,9 +225,11 @@ class KVCache:
         n = len(slot_ids)
         ids = (ctypes.c_int32 * n)(*slot_ids)
         cs = self.c_struct()
+        ws = workspace(q.device) if ws is None else ws
         N.check(N.lib().nvfp4_window_attention(ctypes.byref(cs), ids, n, q.data_ptr(), q.stride(0),
                                                q.shape[0], float(scale), out.data_ptr(),
-                                               out.stride(0), _stream()),
+                                               out.stride(0), ws.data_ptr(), ws.numel(),
+                                               _stream()),
                 "nvfp4_window_attention")
         return out
 

@@ -175,25 +175,29 @@ def test_window_attention_rejects(L):
     f = L.nvfp4_window_attention
     S = ctypes.c_int32 * 3
     ids = S(0, 1, 2)
-    ok = (ids, 3, FAKE, 9216, 2640, 0.088, FAKE, 3072, None)
+    ok = (ids, 3, FAKE, 9216, 2640, 0.088, FAKE, 3072, FAKE, 256, None)
     # argument checks run before any device query, so a call that passes them
     # would reach the device: only failing combinations are exercised here
     assert f(ctypes.byref(c), S(0, 1, 12), 3, *ok[2:]) == N.ERR_INVALID_ARG  # slot out of range
     assert f(ctypes.byref(c), ids, 0, *ok[2:]) == N.ERR_INVALID_ARG
     assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 2640, 0.0, FAKE, 3072,
-             None) == N.ERR_INVALID_ARG  # scale
+             FAKE, 256, None) == N.ERR_INVALID_ARG  # scale
     assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 2640, float("nan"), FAKE, 3072,
-             None) == N.ERR_INVALID_ARG
+             FAKE, 256, None) == N.ERR_INVALID_ARG
     assert f(ctypes.byref(c), ids, 3, FAKE, 3000, 2640, 0.088, FAKE, 3072,
-             None) == N.ERR_INVALID_ARG  # q stride below heads * head_dim
+             FAKE, 256, None) == N.ERR_INVALID_ARG  # q stride below heads * head_dim
     assert f(ctypes.byref(_cache(hd=64)), ids, 3, FAKE, 9216, 2640, 0.088, FAKE, 3072,
-             None) == N.ERR_UNSUPPORTED_SHAPE  # head_dim 128 only
+             FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # head_dim 128 only
     assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 0, 0.088, FAKE, 3072,
-             None) == N.ERR_UNSUPPORTED_SHAPE  # tq
+             FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # tq
     assert f(ctypes.byref(c), ids, 3, FAKE + 8, 9216, 2640, 0.088, FAKE, 3072,
-             None) == N.ERR_MISALIGNED
+             FAKE, 256, None) == N.ERR_MISALIGNED
     assert f(ctypes.byref(c), ids, 3, FAKE, 9220, 2640, 0.088, FAKE, 3072,
-             None) == N.ERR_MISALIGNED
+             FAKE, 256, None) == N.ERR_MISALIGNED
+    assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 2640, 0.088, FAKE, 3072,
+             None, 256, None) == N.ERR_WORKSPACE
+    assert f(ctypes.byref(c), ids, 3, FAKE, 9216, 2640, 0.088, FAKE, 3072,
+             FAKE, 128, None) == N.ERR_WORKSPACE
 
 
 def test_sink_plan_null_and_bad_arguments(L):
