@@ -516,6 +516,11 @@ def run_case(args) -> int:
         qw = nv.quantize((torch.randn(n, k, device=dev, generator=g) * 0.02).to(torch.bfloat16))
         out = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
         run = lambda: nv.gemm(qa, qw, out=out, ws=ws, act=act)  # noqa: E731
+    elif case == "quant_fused":
+        x = torch.randn(M, D, device=dev, generator=g).to(torch.bfloat16)
+        q = nv.empty(M, D, device=dev)
+        # no tensor scale handed in: amax and codes in one pass over the tensor
+        run = lambda: nv.quantize(x, out=q, ws=ws)  # noqa: E731
     elif case in ("quant_act", "quant_ffn"):
         cols = D if case == "quant_act" else F
         x = torch.randn(M, cols, device=dev, generator=g).to(torch.bfloat16)
@@ -730,7 +735,7 @@ def run_ours(args):
                 "vs_onto_6_us": kernel_ms["kv_quant"] / args.layers * 1e3},
             "window_attention": {
                 "us": attn_ms * 1e3, "tflops": ATTN_FLOPS / (attn_ms * 1e-3) / 1e12,
-                "bound": "tensor (bf16 mma.sync)",
+                "bound": "tensor (bf16 tcgen05.mma, fp32 accumulate in tensor memory)",
                 "frac_bf16_peak": ATTN_FLOPS / (attn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                 "shape": f"{M} queries x {WINDOW * TPF} keys x {wl.HEADS} heads x {wl.HEAD_DIM}"},
             "gemm": {"tflops": gemm_tflops, "ms_per_step": gemm_ms,
@@ -771,7 +776,7 @@ def main():
                     help="skip the single-call workload timings and the library comparison")
     ap.add_argument("--case", default=None,
                     help="profiling: run one kernel on a step-shaped case --reps times "
-                         "(gemm_qkv gemm_out gemm_up gemm_down quant_act quant_ffn kv_quant "
+                         "(gemm_qkv gemm_out gemm_up gemm_down quant_act quant_ffn quant_fused kv_quant "
                          "kv_quant_fos kv_dequant attention)")
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()

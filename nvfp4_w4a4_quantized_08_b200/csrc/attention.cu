@@ -15,34 +15,37 @@
 // over the window's tokens j in slot-list order; no mask inside the window
 // (chunk-wise attention: the chunk sees itself and the cached frames whole).
 //
-// Structure: one CTA per (128 queries, head), 13 warps.
-//   warps 0..3  softmax and epilogue: warp w owns tensor-memory lane quadrant
-//               w, i.e. query rows 32w..32w+31, one row per thread.  They load
-//               Q into shared memory once; per KV tile they read the scores
-//               S = Q K^T of their row out of tensor memory, update the running
-//               row maximum and sum (base 2), and write the probabilities
-//               rounded to bf16 back into tensor memory, where the P V product
-//               reads them as its A operand.
-//   warp 4      tensor-memory owner; lane 0 issues the MMAs
-//               (tcgen05.mma kind::f16, bf16 in, fp32 accumulate):
-//               S_j = Q K_j^T into one of three score buffers, then
-//               O += P_{j-1} V_{j-1}, so the tensor core computes the next
-//               tile's scores while the softmax warps work on the current one.
-//   warps 5..12 decoders: per 128-token tile, the 16-element NVFP4 blocks of
+// Structure: one CTA per (256 queries, head): two query tiles of 128 rows (Q0,
+// Q1) share every decoded K/V tile, so a tile is decoded once per 256 queries;
+// 17 warps.
+//   warps 0..7  softmax and epilogue: group g = warp / 4 owns query tile g,
+//               warp w owns tensor-memory lane quadrant w % 4 (one query row
+//               per thread).  They load their Q rows into shared memory once;
+//               per KV tile they read their row of S_g = Q_g K^T out of tensor
+//               memory, update the running row maximum and sum (base 2), and
+//               write the probabilities rounded to bf16 back over S_g, where
+//               the P V product reads them as its A operand.
+//   warp 8      tensor-memory owner; lane 0 issues the MMAs
+//               (tcgen05.mma kind::f16, bf16 in, fp32 accumulate) so that the
+//               tensor core works on one query tile while the other's
+//               softmax runs: ... PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, PV0_{j+1} ...
+//               (each S writes the tensor memory the preceding P V of the same
+//               tile read; the tensor core runs one thread's MMAs in order).
+//   warps 9..16 decoders: per 128-token tile, the 16-element NVFP4 blocks of
 //               K and V of this head -> bf16 (byte-permute table per block),
 //               K as [token][dim] and V transposed as [dim][token], both in
 //               the tensor core's 128-byte-swizzled K-major layout, into a
-//               two-stage ring.
-// Tensor memory (512 columns): O in [0,128), three score buffers at 128, 256
-// and 384; tile j's scores (then its probabilities) use buffer j % 3, and the
-// issuer writes a buffer again only after the P V product that read it has
-// completed (p_free), which with three buffers it almost never waits for.
+//               two-stage ring; each decoder loads the next tile's NVFP4
+//               bytes into registers before it decodes the current one, so
+//               the L2 latency of those loads hides behind the decoding.
+// Tensor memory (512 columns): O0, O1, S0, S1 at columns 0, 128, 256, 384.
 // The running maximum is raised lazily: while a row's new scores stay within
 // 2^8 of the maximum in use, the probabilities are taken against the old one
-// (they stay <= 2^8); only a larger step rescales the row's O and sum, after
-// the previous P V product has completed.  Every wait is bounded: one that
-// runs out records NVFP4_ERR_TIMEOUT in the workspace status word, and the CTA
-// drains its MMAs, frees tensor memory and returns.
+// (they stay <= 2^8); only a larger step rescales the row's O and sum, which
+// is safe at once: S_g of tile j completes after P V of tile j-1 of the same
+// query tile.  Every wait is bounded: one that runs out records
+// NVFP4_ERR_TIMEOUT in the workspace status word, and the CTA drains its MMAs,
+// frees tensor memory and returns.
 #include "common.cuh"
 #include "decode.cuh"
 #include "kernels.h"
@@ -53,32 +56,32 @@ namespace nvfp4 {
 namespace attn {
 
 constexpr int kD = 128;                   // head_dim
-constexpr int kBQ = 128;                  // queries per CTA (tensor-memory lanes)
+constexpr int kBQ = 128;                  // queries per query tile (tensor-memory lanes)
+constexpr int kQTiles = 2;                // query tiles per CTA
 constexpr int kBK = 128;                  // keys per tile
 constexpr int kDimBlocks = kD / 16;       // 16-element blocks per token and head
-constexpr int kSoftWarps = 4;             // warps 0..3
-constexpr int kMmaWarp = 4;
-constexpr int kDecWarp0 = 5;
+constexpr int kSoftWarps = 4 * kQTiles;   // warps 0..7
+constexpr int kMmaWarp = kSoftWarps;      // 8
+constexpr int kDecWarp0 = kMmaWarp + 1;   // 9
 constexpr int kDecWarps = 8;
-constexpr int kThreads = (kDecWarp0 + kDecWarps) * 32;  // 416
+constexpr int kThreads = (kDecWarp0 + kDecWarps) * 32;  // 544
 constexpr int kStages = 2;
 constexpr int kChunkBytes = 128 * 128;    // 128 rows x 64 bf16 (one K chunk of an operand)
 constexpr int kOpBytes = 2 * kChunkBytes;  // 128 rows x 128 bf16
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kOpBytes;                // + stage * kOpBytes
-constexpr int kOffV = kOffK + kStages * kOpBytes;      // transposed V, + stage * kOpBytes
+constexpr int kOffQ = 0;                                 // + g * kOpBytes
+constexpr int kOffK = kOffQ + kQTiles * kOpBytes;        // + stage * kOpBytes
+constexpr int kOffV = kOffK + kStages * kOpBytes;        // transposed V, + stage * kOpBytes
 constexpr int kOffBar = kOffV + kStages * kOpBytes;
-// q_ready, kv_full[2], kv_empty[2], s_full[3], p_ready[3], p_free[3], pv_done, o_full, drain
-constexpr int kSBufs = 3;
-constexpr int kNumBars = 1 + 2 * kStages + 3 * kSBufs + 3;
+// q_ready, kv_full[2], kv_empty[2], s_full[2], p_ready[2], pv_done[2], o_full, drain
+constexpr int kNumBars = 1 + 2 * kStages + 3 * kQTiles + 2;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
 constexpr int kSmemBytes = kOffAbort + 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 0;
-constexpr uint32_t kSCol0 = 128;          // score buffer b at kSCol0 + 128 b
+constexpr uint32_t kOCol0 = 0;            // O_g at kOCol0 + 128 g
+constexpr uint32_t kSCol0 = 256;          // S_g (then P_g) at kSCol0 + 128 g
 // Instruction descriptor, kind::f16: fp32 D (bit 4), bf16 A and B (bits 7 and
 // 10), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBK >> 3) << 17) |
@@ -174,6 +177,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// The same load without its wait (pair with tmem_wait_ld).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -210,6 +229,14 @@ __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
 // 128-byte-swizzled layout (two 64-element chunks of 16 KB).
 __device__ __forceinline__ uint32_t op_offset(uint32_t r, uint32_t u) {
   return (u >> 3) * kChunkBytes + (r >> 3) * 1024 + (r & 7) * 128 + (((u & 7) ^ (r & 7)) << 4);
+}
+
+// 2^x with the hardware approximation (relative error about 2^-22; results
+// below 2^-126 flush to zero, which the softmax sums cannot notice).
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 struct Waiter {
@@ -255,18 +282,17 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
   const uint32_t bar_q = sbase + kOffBar;
   const uint32_t bar_kv_full = bar_q + 8;                      // + 8 stage
   const uint32_t bar_kv_empty = bar_kv_full + 8 * kStages;     // + 8 stage
-  const uint32_t bar_s_full = bar_kv_empty + 8 * kStages;      // + 8 buffer
-  const uint32_t bar_p_ready = bar_s_full + 8 * kSBufs;        // + 8 buffer
-  const uint32_t bar_p_free = bar_p_ready + 8 * kSBufs;        // + 8 buffer
-  const uint32_t bar_pv_done = bar_p_free + 8 * kSBufs;
-  const uint32_t bar_o_full = bar_pv_done + 8;
+  const uint32_t bar_s_full = bar_kv_empty + 8 * kStages;      // + 8 g
+  const uint32_t bar_p_ready = bar_s_full + 8 * kQTiles;       // + 8 g
+  const uint32_t bar_pv_done = bar_p_ready + 8 * kQTiles;      // + 8 g
+  const uint32_t bar_o_full = bar_pv_done + 8 * kQTiles;
   const uint32_t bar_drain = bar_o_full + 8;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t h = blockIdx.y;
-  const uint32_t q0 = blockIdx.x * kBQ;
+  const uint32_t q_base = blockIdx.x * (kBQ * kQTiles);
   const uint32_t n_tiles = (a.n_kv + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
@@ -275,12 +301,11 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
       bar_init(bar_kv_full + 8 * s, kDecWarps);
       bar_init(bar_kv_empty + 8 * s, 1);
     }
-    for (int b = 0; b < kSBufs; ++b) {
-      bar_init(bar_s_full + 8 * b, 1);
-      bar_init(bar_p_ready + 8 * b, kSoftWarps);
-      bar_init(bar_p_free + 8 * b, 1);
+    for (int g = 0; g < kQTiles; ++g) {
+      bar_init(bar_s_full + 8 * g, 1);
+      bar_init(bar_p_ready + 8 * g, 4);
+      bar_init(bar_pv_done + 8 * g, 1);
     }
-    bar_init(bar_pv_done, 1);
     bar_init(bar_o_full, 1);
     bar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -303,17 +328,23 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
 
   if (warp < kSoftWarps) {
     // ------------------------------------------------------------ softmax
-    const uint32_t row = uint32_t(warp) * 32 + uint32_t(lane);   // query row of this thread
-    const uint32_t lane_bits = (uint32_t(warp) * 32) << 16;
+    const uint32_t g = uint32_t(warp) >> 2;                      // query tile
+    const uint32_t quad = uint32_t(warp) & 3;                    // lane quadrant
+    const uint32_t row = quad * 32 + uint32_t(lane);             // row within the tile
+    const uint32_t q0 = q_base + g * kBQ;
+    const uint32_t lane_bits = (quad * 32) << 16;
+    const uint32_t o_addr = tmem + lane_bits + kOCol0 + 128 * g;
+    const uint32_t s_addr = tmem + lane_bits + kSCol0 + 128 * g;
     // Q row -> shared memory (rows past tq are zero)
     {
       const bool live = q0 + row < a.tq;
       const uint4* src =
-          reinterpret_cast<const uint4*>(a.q + int64_t(q0 + (live ? row : 0)) * a.q_stride + h * kD);
+          reinterpret_cast<const uint4*>(a.q + int64_t(live ? q0 + row : 0) * a.q_stride + h * kD);
+      const uint32_t qs = sbase + kOffQ + g * kOpBytes;
 #pragma unroll
       for (uint32_t u = 0; u < 16; ++u) {
         const uint4 v = live ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
-        st_shared_v4(sbase + kOffQ + op_offset(row, u), v);
+        st_shared_v4(qs + op_offset(row, u), v);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
@@ -322,32 +353,44 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (uint32_t j = 0; j < n_tiles && ok; ++j) {
-      const uint32_t b = j % kSBufs;
-      ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_s_full + 8 * b, (j / kSBufs) & 1));
+      ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_s_full + 8 * g, j & 1));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_bits + kSCol0 + 128 * b;
       const uint32_t n_valid = min(uint32_t(kBK), a.n_kv - j * kBK);
-      // pass 1: the tile's row maximum (scaled, base 2) over the live keys
-      float mx = -INFINITY;
+      // pass 1: the tile's row maximum over the live keys (the scale is
+      // positive, so scaling the maximum is the maximum of the scaled scores)
+      float mx_raw = -INFINITY;
+      const bool tail = n_valid < uint32_t(kBK);
 #pragma unroll 1
-      for (uint32_t c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_addr + 32 * c, r);
+      for (uint32_t c = 0; c < 4; c += 2) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32_async(s_addr + 32 * c, r0);
+        tmem_ld32_async(s_addr + 32 * c + 32, r1);
+        tmem_wait_ld();
+        if (!tail) {
 #pragma unroll
-        for (uint32_t e = 0; e < 32; ++e)
-          if (32 * c + e < n_valid) mx = fmaxf(mx, __fmul_rn(__uint_as_float(r[e]), a.scale_log2));
+          for (uint32_t e = 0; e < 32; ++e)
+            mx_raw = fmaxf(mx_raw, fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
+        } else {
+#pragma unroll
+          for (uint32_t e = 0; e < 32; ++e) {
+            if (32 * c + e < n_valid) mx_raw = fmaxf(mx_raw, __uint_as_float(r0[e]));
+            if (32 * c + 32 + e < n_valid) mx_raw = fmaxf(mx_raw, __uint_as_float(r1[e]));
+          }
+        }
       }
+      const float mx = __fmul_rn(mx_raw, a.scale_log2);
       // lazy maximum: keep the one in use while the tile stays within 2^8 of it
       float factor = 1.0f;
       if (mx > m_run + kLazyLog2) {
-        factor = exp2f(m_run - mx);   // 0 on the first tile
+        factor = exp2_approx(m_run - mx);   // 0 on the first tile
         m_run = mx;
         l_run = l_run * factor;
       }
-      // pass 2: probabilities, their sum, bf16 into the score buffer's first
-      // 64 columns (chunk c's 16 words go over columns already read)
-      float sum = 0.0f;
+      // pass 2: probabilities 2^(s scale - m), their sum, bf16 into the score
+      // buffer's first 64 columns (chunk c's 16 words go over columns already read)
+      const float neg_m = -m_run;
+      float sum0 = 0.0f, sum1 = 0.0f;
 #pragma unroll 1
       for (uint32_t c = 0; c < 4; ++c) {
         uint32_t r[32];
@@ -356,38 +399,40 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
 #pragma unroll
         for (uint32_t e = 0; e < 16; ++e) {
           const uint32_t k0 = 32 * c + 2 * e;
-          const float p0 = k0 < n_valid
-                               ? exp2f(__fmul_rn(__uint_as_float(r[2 * e]), a.scale_log2) - m_run)
-                               : 0.0f;
-          const float p1 = k0 + 1 < n_valid
-                               ? exp2f(__fmul_rn(__uint_as_float(r[2 * e + 1]), a.scale_log2) - m_run)
-                               : 0.0f;
-          sum += p0 + p1;
+          float p0 = exp2_approx(__fmaf_rn(__uint_as_float(r[2 * e]), a.scale_log2, neg_m));
+          float p1 = exp2_approx(__fmaf_rn(__uint_as_float(r[2 * e + 1]), a.scale_log2, neg_m));
+          if (tail) {
+            p0 = k0 < n_valid ? p0 : 0.0f;
+            p1 = k0 + 1 < n_valid ? p1 : 0.0f;
+          }
+          sum0 += p0;
+          sum1 += p1;
           pk[e] = bf16x2_rn(p0, p1);
         }
         tmem_st16(s_addr + 16 * c, pk);
       }
-      l_run += sum;
-      // a raised maximum rescales this row's O, once the previous P V is done
+      l_run += sum0 + sum1;
+      // a raised maximum rescales this row's O (tile j-1's P V, complete since
+      // S_g of tile j is)
       if (__any_sync(0xFFFFFFFFu, factor != 1.0f) && j > 0) {
-        ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_pv_done, (j - 1) & 1));
+        ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_pv_done + 8 * g, (j - 1) & 1));
         if (ok) {
           tc_fence_after();
 #pragma unroll 1
           for (uint32_t c = 0; c < 4; ++c) {
             uint32_t r[32];
-            tmem_ld32(tmem + lane_bits + kOCol + 32 * c, r);
+            tmem_ld32(o_addr + 32 * c, r);
 #pragma unroll
             for (uint32_t e = 0; e < 32; ++e)
               r[e] = __float_as_uint(__fmul_rn(__uint_as_float(r[e]), factor));
-            tmem_st32(tmem + lane_bits + kOCol + 32 * c, r);
+            tmem_st32(o_addr + 32 * c, r);
           }
         }
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) bar_arrive(bar_p_ready + 8 * b);
+      if (lane == 0) bar_arrive(bar_p_ready + 8 * g);
     }
     // ---- epilogue: O / l -> bf16 (rows past tq are not stored)
     if (ok) ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_o_full, 0));
@@ -395,11 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const bool live = q0 + row < a.tq;
-      uint4* dst = reinterpret_cast<uint4*>(a.out + int64_t(q0 + row) * a.out_stride + h * kD);
+      uint4* dst = reinterpret_cast<uint4*>(a.out + int64_t(live ? q0 + row : 0) * a.out_stride +
+                                            h * kD);
 #pragma unroll 1
       for (uint32_t c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_bits + kOCol + 32 * c, r);
+        tmem_ld32(o_addr + 32 * c, r);
         if (live) {
 #pragma unroll
           for (uint32_t e = 0; e < 4; ++e) {
@@ -417,41 +463,51 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = waiter.wait(bar_q, 0);
-      const uint64_t qd = desc_sw128(sbase + kOffQ);
-      // O += P_jj V_jj: P from score buffer jj % 3, V^T from ring stage jj % 2
-      auto issue_pv = [&](uint32_t jj) {
-        const uint32_t bb = jj % kSBufs, st = jj % kStages;
-        if (!waiter.wait(bar_p_ready + 8 * bb, (jj / kSBufs) & 1)) return false;
-        tc_fence_after();
-        const uint64_t vd = desc_sw128(sbase + kOffV + st * kOpBytes);
-        const uint32_t p_addr = tmem + kSCol0 + 128 * bb;
-#pragma unroll
-        for (uint32_t ks = 0; ks < 8; ++ks)  // 16 keys a step: 8 columns of P, 32 bytes of V^T
-          mma_ts(tmem + kOCol, p_addr + 8 * ks,
-                 vd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3), (jj | ks) != 0);
-        tc_commit(bar_kv_empty + 8 * st);
-        tc_commit(bar_p_free + 8 * bb);
-        tc_commit(bar_pv_done);
-        return true;
-      };
-      for (uint32_t j = 0; j < n_tiles && ok; ++j) {
-        const uint32_t st = j % kStages, b = j % kSBufs;
-        if (!waiter.wait(bar_kv_full + 8 * st, (j / kStages) & 1)) { ok = false; break; }
-        // the P V product that last read score buffer b (tile j - 3) is done
-        if (j >= kSBufs && !waiter.wait(bar_p_free + 8 * b, (j / kSBufs - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      // S_g(j) = Q_g K_j^T into S_g
+      auto issue_s = [&](uint32_t g, uint32_t j) {
+        const uint32_t st = j % kStages;
+        const uint64_t qd = desc_sw128(sbase + kOffQ + g * kOpBytes);
         const uint64_t kd = desc_sw128(sbase + kOffK + st * kOpBytes);
 #pragma unroll
         for (uint32_t ks = 0; ks < 8; ++ks)  // 16 dims a step: +32 bytes, next chunk after 4
-          mma_ss(tmem + kSCol0 + 128 * b, qd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3),
+          mma_ss(tmem + kSCol0 + 128 * g, qd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3),
                  kd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3), ks != 0);
-        tc_commit(bar_s_full + 8 * b);
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+        tc_commit(bar_s_full + 8 * g);
+      };
+      // O_g += P_g(j) V_j, P from S_g's columns, V^T from ring stage j % 2
+      auto issue_pv = [&](uint32_t g, uint32_t j) {
+        if (!waiter.wait(bar_p_ready + 8 * g, j & 1)) return false;
+        tc_fence_after();
+        const uint64_t vd = desc_sw128(sbase + kOffV + (j % kStages) * kOpBytes);
+        const uint32_t p_addr = tmem + kSCol0 + 128 * g;
+#pragma unroll
+        for (uint32_t ks = 0; ks < 8; ++ks)  // 16 keys a step: 8 columns of P, 32 bytes of V^T
+          mma_ts(tmem + kOCol0 + 128 * g, p_addr + 8 * ks,
+                 vd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3), (j | ks) != 0);
+        tc_commit(bar_pv_done + 8 * g);
+        return true;
+      };
+      auto kv_ready = [&](uint32_t j) {
+        if (!waiter.wait(bar_kv_full + 8 * (j % kStages), (j / kStages) & 1)) return false;
+        tc_fence_after();
+        return true;
+      };
+      if (ok && n_tiles > 0 && (ok = kv_ready(0))) {
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
-      if (ok && issue_pv(n_tiles - 1)) tc_commit(bar_o_full);
+      for (uint32_t j = 0; j < n_tiles && ok; ++j) {
+        const bool more = j + 1 < n_tiles;
+        if (!(ok = issue_pv(0, j))) break;
+        if (more) {
+          if (!(ok = kv_ready(j + 1))) break;
+          issue_s(0, j + 1);
+        }
+        if (!(ok = issue_pv(1, j))) break;
+        tc_commit(bar_kv_empty + 8 * (j % kStages));   // K_j and V_j read by every MMA
+        if (more) issue_s(1, j + 1);
+      }
+      if (ok) tc_commit(bar_o_full);
       // drain: every tcgen05 operation this thread issued has completed
       tc_commit(bar_drain);
       const uint64_t t0 = globaltimer();
@@ -465,39 +521,48 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
     __syncwarp();
   } else {
     // ------------------------------------------------------------ decoders
+    // K: token t / 8 + 32 i, dim block t % 8 (8 lanes read one token's 64
+    // bytes); V: token pair p = t % 64 (tokens 2p, 2p + 1), dim block
+    // t / 64 + 4 i (a warp's transposed stores then fill whole 128-byte rows)
     const uint32_t t = threadIdx.x - kDecWarp0 * 32;   // 0..255
-    bool ok = true;
-    for (uint32_t j = 0; j < n_tiles && ok; ++j) {
-      const uint32_t b = j % kStages;
-      ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_kv_empty + 8 * b, ((j / kStages) & 1) ^ 1));
-      if (!ok) break;
-      const uint32_t w0 = j * kBK;
-      // K: token t / 8 + 32 i, dim block t % 8 (8 lanes read one token's 64 bytes)
+    const uint32_t p = t % 64;
+    struct TileRaw {
       uint2 kc[4];
       uint32_t ksb[4];
       float kst[4];
-#pragma unroll
-      for (uint32_t i = 0; i < 4; ++i)
-        load_block(a, 0, w0 + t / 8 + 32 * i, h, t % 8, kc[i], ksb[i], kst[i]);
-      // V: token pair p = t % 64 (tokens 2p, 2p + 1), dim block t / 64 + 4 i
       uint2 vc[2][2];
       uint32_t vsb[2][2];
       float vst[2][2];
-      const uint32_t p = t % 64;
+    };
+    auto load_tile = [&](uint32_t j, TileRaw& r) {
+      const uint32_t w0 = j * kBK;
+#pragma unroll
+      for (uint32_t i = 0; i < 4; ++i)
+        load_block(a, 0, w0 + t / 8 + 32 * i, h, t % 8, r.kc[i], r.ksb[i], r.kst[i]);
 #pragma unroll
       for (uint32_t i = 0; i < 2; ++i)
 #pragma unroll
         for (uint32_t e = 0; e < 2; ++e)
-          load_block(a, 1, w0 + 2 * p + e, h, t / 64 + 4 * i, vc[i][e], vsb[i][e], vst[i][e]);
+          load_block(a, 1, w0 + 2 * p + e, h, t / 64 + 4 * i, r.vc[i][e], r.vsb[i][e], r.vst[i][e]);
+    };
+    TileRaw cur, nxt;
+    if (n_tiles > 0) load_tile(0, cur);
+    bool ok = true;
+    for (uint32_t j = 0; j < n_tiles && ok; ++j) {
+      if (j + 1 < n_tiles) load_tile(j + 1, nxt);
+      const uint32_t b = j % kStages;
+      ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_kv_empty + 8 * b, ((j / kStages) & 1) ^ 1));
+      if (!ok) break;
+      const uint32_t w0 = j * kBK;
       const uint32_t kbase = sbase + kOffK + b * kOpBytes;
 #pragma unroll
       for (uint32_t i = 0; i < 4; ++i) {
         const uint32_t tok = t / 8 + 32 * i, db = t % 8;
         uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
         if (w0 + tok < a.n_kv) {
-          const BlockLut l = make_lut(ksb[i], kst[i]);
-          lo = decode8(l, kc[i].x);
-          hi = decode8(l, kc[i].y);
+          const BlockLut l = make_lut(cur.ksb[i], cur.kst[i]);
+          lo = decode8(l, cur.kc[i].x);
+          hi = decode8(l, cur.kc[i].y);
         }
         st_shared_v4(kbase + op_offset(tok, 2 * db), lo);
         st_shared_v4(kbase + op_offset(tok, 2 * db + 1), hi);
@@ -511,9 +576,9 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
         for (uint32_t e = 0; e < 2; ++e) {
           uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
           if (w0 + 2 * p + e < a.n_kv) {
-            const BlockLut l = make_lut(vsb[i][e], vst[i][e]);
-            lo = decode8(l, vc[i][e].x);
-            hi = decode8(l, vc[i][e].y);
+            const BlockLut l = make_lut(cur.vsb[i][e], cur.vst[i][e]);
+            lo = decode8(l, cur.vc[i][e].x);
+            hi = decode8(l, cur.vc[i][e].y);
           }
           wv[e][0] = lo.x; wv[e][1] = lo.y; wv[e][2] = lo.z; wv[e][3] = lo.w;
           wv[e][4] = hi.x; wv[e][5] = hi.y; wv[e][6] = hi.z; wv[e][7] = hi.w;
@@ -529,6 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) bar_arrive(bar_kv_full + 8 * b);
+      cur = nxt;
     }
   }
 
@@ -575,7 +641,8 @@ cudaError_t launch_window_attention(const LaunchAttn& d, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured[dev].store(true, std::memory_order_release);
   }
-  const dim3 grid(uint32_t((d.tq + attn::kBQ - 1) / attn::kBQ), uint32_t(d.heads));
+  constexpr int64_t kCtaQ = int64_t(attn::kBQ) * attn::kQTiles;
+  const dim3 grid(uint32_t((d.tq + kCtaQ - 1) / kCtaQ), uint32_t(d.heads));
   return launch_pdl(attn::window_attention_kernel, grid, dim3(attn::kThreads),
                     size_t(attn::kSmemBytes), st, a);
 }
