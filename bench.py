@@ -516,10 +516,10 @@ def run_case(args) -> int:
         qw = nv.quantize((torch.randn(n, k, device=dev, generator=g) * 0.02).to(torch.bfloat16))
         out = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
         run = lambda: nv.gemm(qa, qw, out=out, ws=ws, act=act)  # noqa: E731
-    elif case == "quant_fused":
+    elif case == "quant_amax":
         x = torch.randn(M, D, device=dev, generator=g).to(torch.bfloat16)
         q = nv.empty(M, D, device=dev)
-        # no tensor scale handed in: amax and codes in one pass over the tensor
+        # no tensor scale handed in: the amax pass, then the encode
         run = lambda: nv.quantize(x, out=q, ws=ws)  # noqa: E731
     elif case in ("quant_act", "quant_ffn"):
         cols = D if case == "quant_act" else F
@@ -776,7 +776,7 @@ def main():
                     help="skip the single-call workload timings and the library comparison")
     ap.add_argument("--case", default=None,
                     help="profiling: run one kernel on a step-shaped case --reps times "
-                         "(gemm_qkv gemm_out gemm_up gemm_down quant_act quant_ffn quant_fused kv_quant "
+                         "(gemm_qkv gemm_out gemm_up gemm_down quant_act quant_ffn quant_amax kv_quant "
                          "kv_quant_fos kv_dequant attention)")
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()

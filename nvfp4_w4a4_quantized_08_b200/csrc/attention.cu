@@ -33,9 +33,10 @@
 //               tile read; the tensor core runs one thread's MMAs in order).
 //   warps 9..16 decoders: per 128-token tile, the 16-element NVFP4 blocks of
 //               K and V of this head -> bf16 (byte-permute table per block),
-//               K as [token][dim] and V transposed as [dim][token], both in
-//               the tensor core's 128-byte-swizzled K-major layout, into a
-//               two-stage ring; each decoder loads the next tile's NVFP4
+//               K and V both as [token][dim] in the tensor core's
+//               128-byte-swizzled layout (K-major for S = Q K^T; for P V the
+//               same bytes are V in the MN-major layout), into a two-stage
+//               ring; each decoder loads the next tile's NVFP4
 //               bytes into registers before it decodes the current one, so
 //               the L2 latency of those loads hides behind the decoding.
 // Tensor memory (512 columns): O0, O1, S0, S1 at columns 0, 128, 256, 384.
@@ -71,7 +72,7 @@ constexpr int kOpBytes = 2 * kChunkBytes;  // 128 rows x 128 bf16
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffQ = 0;                                 // + g * kOpBytes
 constexpr int kOffK = kOffQ + kQTiles * kOpBytes;        // + stage * kOpBytes
-constexpr int kOffV = kOffK + kStages * kOpBytes;        // transposed V, + stage * kOpBytes
+constexpr int kOffV = kOffK + kStages * kOpBytes;        // V [token][dim], + stage * kOpBytes
 constexpr int kOffBar = kOffV + kStages * kOpBytes;
 // q_ready, kv_full[2], kv_empty[2], s_full[2], p_ready[2], pv_done[2], o_full, drain
 constexpr int kNumBars = 1 + 2 * kStages + 3 * kQTiles + 2;
@@ -155,13 +156,29 @@ __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint3
       "l"(a), "l"(b), "r"(kIdesc), "r"(acc)
       : "memory");
 }
-// D (+)= A B^T, A in tensor memory.
+// Shared-memory matrix descriptor of an MN-major operand, 128-byte swizzle:
+// 8-row (K) groups 1024 bytes apart (SBO), 64-element MN chunks
+// kMnChunkBytes apart (LBO), descriptor version 1.
+#ifndef ATTN_V_LBO
+#define ATTN_V_LBO (128 * 128)
+#endif
+#ifndef ATTN_V_SBO
+#define ATTN_V_SBO 1024
+#endif
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t addr) {
+  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t(ATTN_V_LBO >> 4) << 16) |
+         (uint64_t(ATTN_V_SBO >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// The P V product's descriptor: as kIdesc with B MN-major (bit 16): V is
+// stored [key][dim], dims contiguous.
+constexpr uint32_t kIdescPV = kIdesc | (1u << 16);
+// D (+)= A B^T, A in tensor memory, B MN-major.
 __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a), "l"(b), "r"(kIdesc), "r"(acc)
+      "r"(a), "l"(b), "r"(kIdescPV), "r"(acc)
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -392,24 +409,32 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
       const float neg_m = -m_run;
       float sum0 = 0.0f, sum1 = 0.0f;
 #pragma unroll 1
-      for (uint32_t c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_addr + 32 * c, r);
-        uint32_t pk[16];
+      for (uint32_t c = 0; c < 4; c += 2) {
+        // two 32-column chunks per tensor-memory round trip
+        uint32_t r[2][32];
+        tmem_ld32_async(s_addr + 32 * c, r[0]);
+        tmem_ld32_async(s_addr + 32 * c + 32, r[1]);
+        tmem_wait_ld();
 #pragma unroll
-        for (uint32_t e = 0; e < 16; ++e) {
-          const uint32_t k0 = 32 * c + 2 * e;
-          float p0 = exp2_approx(__fmaf_rn(__uint_as_float(r[2 * e]), a.scale_log2, neg_m));
-          float p1 = exp2_approx(__fmaf_rn(__uint_as_float(r[2 * e + 1]), a.scale_log2, neg_m));
-          if (tail) {
-            p0 = k0 < n_valid ? p0 : 0.0f;
-            p1 = k0 + 1 < n_valid ? p1 : 0.0f;
+        for (uint32_t h2 = 0; h2 < 2; ++h2) {
+          uint32_t pk[16];
+#pragma unroll
+          for (uint32_t e = 0; e < 16; ++e) {
+            const uint32_t k0 = 32 * (c + h2) + 2 * e;
+            float p0 = exp2_approx(__fmaf_rn(__uint_as_float(r[h2][2 * e]), a.scale_log2, neg_m));
+            float p1 =
+                exp2_approx(__fmaf_rn(__uint_as_float(r[h2][2 * e + 1]), a.scale_log2, neg_m));
+            if (tail) {
+              p0 = k0 < n_valid ? p0 : 0.0f;
+              p1 = k0 + 1 < n_valid ? p1 : 0.0f;
+            }
+            sum0 += p0;
+            sum1 += p1;
+            pk[e] = bf16x2_rn(p0, p1);
           }
-          sum0 += p0;
-          sum1 += p1;
-          pk[e] = bf16x2_rn(p0, p1);
+          // P chunk c + h2 -> columns 16 (c + h2): inside chunks already read
+          tmem_st16(s_addr + 16 * (c + h2), pk);
         }
-        tmem_st16(s_addr + 16 * c, pk);
       }
       l_run += sum0 + sum1;
       // a raised maximum rescales this row's O (tile j-1's P V, complete since
@@ -474,16 +499,15 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
                  kd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3), ks != 0);
         tc_commit(bar_s_full + 8 * g);
       };
-      // O_g += P_g(j) V_j, P from S_g's columns, V^T from ring stage j % 2
+      // O_g += P_g(j) V_j, P from S_g's columns, V from ring stage j % 2
       auto issue_pv = [&](uint32_t g, uint32_t j) {
         if (!waiter.wait(bar_p_ready + 8 * g, j & 1)) return false;
         tc_fence_after();
-        const uint64_t vd = desc_sw128(sbase + kOffV + (j % kStages) * kOpBytes);
+        const uint64_t vd = desc_mn_sw128(sbase + kOffV + (j % kStages) * kOpBytes);
         const uint32_t p_addr = tmem + kSCol0 + 128 * g;
 #pragma unroll
-        for (uint32_t ks = 0; ks < 8; ++ks)  // 16 keys a step: 8 columns of P, 32 bytes of V^T
-          mma_ts(tmem + kOCol0 + 128 * g, p_addr + 8 * ks,
-                 vd + (ks >> 2) * (kChunkBytes >> 4) + 2 * (ks & 3), (j | ks) != 0);
+        for (uint32_t ks = 0; ks < 8; ++ks)  // 16 keys a step: 8 columns of P, two 8-key groups of V
+          mma_ts(tmem + kOCol0 + 128 * g, p_addr + 8 * ks, vd + ks * (2048 >> 4), (j | ks) != 0);
         tc_commit(bar_pv_done + 8 * g);
         return true;
       };
@@ -521,29 +545,22 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
     __syncwarp();
   } else {
     // ------------------------------------------------------------ decoders
-    // K: token t / 8 + 32 i, dim block t % 8 (8 lanes read one token's 64
-    // bytes); V: token pair p = t % 64 (tokens 2p, 2p + 1), dim block
-    // t / 64 + 4 i (a warp's transposed stores then fill whole 128-byte rows)
+    // K and V alike: token t / 8 + 32 i, dim block t % 8 (8 lanes read one
+    // token's 64 bytes), stored [token][dim]: K-major for S = Q K^T, and the
+    // MN-major layout the P V product reads V in
     const uint32_t t = threadIdx.x - kDecWarp0 * 32;   // 0..255
-    const uint32_t p = t % 64;
     struct TileRaw {
-      uint2 kc[4];
-      uint32_t ksb[4];
-      float kst[4];
-      uint2 vc[2][2];
-      uint32_t vsb[2][2];
-      float vst[2][2];
+      uint2 c[2][4];
+      uint32_t sb[2][4];
+      float st[2][4];
     };
     auto load_tile = [&](uint32_t j, TileRaw& r) {
       const uint32_t w0 = j * kBK;
 #pragma unroll
-      for (uint32_t i = 0; i < 4; ++i)
-        load_block(a, 0, w0 + t / 8 + 32 * i, h, t % 8, r.kc[i], r.ksb[i], r.kst[i]);
+      for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-      for (uint32_t i = 0; i < 2; ++i)
-#pragma unroll
-        for (uint32_t e = 0; e < 2; ++e)
-          load_block(a, 1, w0 + 2 * p + e, h, t / 64 + 4 * i, r.vc[i][e], r.vsb[i][e], r.vst[i][e]);
+        for (uint32_t i = 0; i < 4; ++i)
+          load_block(a, pl, w0 + t / 8 + 32 * i, h, t % 8, r.c[pl][i], r.sb[pl][i], r.st[pl][i]);
     };
     TileRaw cur, nxt;
     if (n_tiles > 0) load_tile(0, cur);
@@ -554,41 +571,20 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
       ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_kv_empty + 8 * b, ((j / kStages) & 1) ^ 1));
       if (!ok) break;
       const uint32_t w0 = j * kBK;
-      const uint32_t kbase = sbase + kOffK + b * kOpBytes;
 #pragma unroll
-      for (uint32_t i = 0; i < 4; ++i) {
-        const uint32_t tok = t / 8 + 32 * i, db = t % 8;
-        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-        if (w0 + tok < a.n_kv) {
-          const BlockLut l = make_lut(cur.ksb[i], cur.kst[i]);
-          lo = decode8(l, cur.kc[i].x);
-          hi = decode8(l, cur.kc[i].y);
-        }
-        st_shared_v4(kbase + op_offset(tok, 2 * db), lo);
-        st_shared_v4(kbase + op_offset(tok, 2 * db + 1), hi);
-      }
-      const uint32_t vbase = sbase + kOffV + b * kOpBytes;
+      for (int pl = 0; pl < 2; ++pl) {
+        const uint32_t base = sbase + (pl == 0 ? kOffK : kOffV) + b * kOpBytes;
 #pragma unroll
-      for (uint32_t i = 0; i < 2; ++i) {
-        const uint32_t db = t / 64 + 4 * i;
-        uint32_t wv[2][8];
-#pragma unroll
-        for (uint32_t e = 0; e < 2; ++e) {
+        for (uint32_t i = 0; i < 4; ++i) {
+          const uint32_t tok = t / 8 + 32 * i, db = t % 8;
           uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-          if (w0 + 2 * p + e < a.n_kv) {
-            const BlockLut l = make_lut(cur.vsb[i][e], cur.vst[i][e]);
-            lo = decode8(l, cur.vc[i][e].x);
-            hi = decode8(l, cur.vc[i][e].y);
+          if (w0 + tok < a.n_kv) {
+            const BlockLut l = make_lut(cur.sb[pl][i], cur.st[pl][i]);
+            lo = decode8(l, cur.c[pl][i].x);
+            hi = decode8(l, cur.c[pl][i].y);
           }
-          wv[e][0] = lo.x; wv[e][1] = lo.y; wv[e][2] = lo.z; wv[e][3] = lo.w;
-          wv[e][4] = hi.x; wv[e][5] = hi.y; wv[e][6] = hi.z; wv[e][7] = hi.w;
-        }
-        // V^T row d = 16 db + k holds keys 2p, 2p + 1 in one word
-#pragma unroll
-        for (uint32_t k = 0; k < 16; ++k) {
-          const uint32_t d = 16 * db + k;
-          const uint32_t word = prmt(wv[0][k >> 1], wv[1][k >> 1], (k & 1) ? 0x7632u : 0x5410u);
-          st_shared_u32(vbase + op_offset(d, p / 4) + (p % 4) * 4, word);
+          st_shared_v4(base + op_offset(tok, 2 * db), lo);
+          st_shared_v4(base + op_offset(tok, 2 * db + 1), hi);
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -814,189 +814,6 @@ __global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4
   check_in(nullptr, amax_in, args.ws, plane);
 }
 
-// ---- one pass for a tensor that fits the grid's shared memory
-// When the tensor scale is not handed in, the recipe needs the whole tensor's
-// amax before any block can be coded.  If the tensor fits in the rings of one
-// resident wave (each CTA's range within its 4 stages), it is read from HBM
-// once: every CTA copies its range in, takes the range's amax, raises the
-// workspace amax word, and waits at a grid-wide barrier (an arrival counter,
-// the grid launched cooperatively so that every CTA is resident) until all
-// CTAs have; then it codes its range straight out of shared memory.  The last
-// CTA to leave resets the counters and the amax word.
-template <typename InT, int kSfLayout>
-__global__ void __launch_bounds__(kTqThreads) quant_fused_kernel(const TmaQuantArgs ta) {
-  constexpr uint32_t kBlockBytes = 16 * sizeof(InT);
-  constexpr uint32_t kStageBlocks = kTqStageBytes / kBlockBytes;
-  const QuantArgs& args = ta.q;
-  extern __shared__ __align__(128) uint8_t fq_smem[];
-  __shared__ float inv_tab[128];
-  __shared__ uint32_t warp_max[kTqConsumers / 32];
-  __shared__ int abort_flag;
-  __shared__ float s_t_shared;
-  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(fq_smem));
-  const uint32_t bar_full = sbase + kTqStages * kTqStageBytes;
-  uint32_t* const status = args.ws + kWsStatus / 4;
-  uint32_t* const amax_word = args.ws + kWsAmax0 / 4;
-  uint32_t* const arrive = args.ws + kWsCount0 / 4;
-  uint32_t* const depart = args.ws + kWsCount1 / 4;
-  fill_inv_table(inv_tab);
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kTqStages; ++s)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_full + 8 * s) : "memory");
-    abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  pdl_wait();
-  pdl_trigger();
-  const uint32_t blocks = args.in.units >> 1;
-  const uint32_t b_lo = blockIdx.x * ta.per_cta;
-  const uint32_t b_hi = min(blocks, b_lo + ta.per_cta);
-  const uint32_t n_stages = b_hi > b_lo ? (b_hi - b_lo + kStageBlocks - 1) / kStageBlocks : 0;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  volatile int* abort = &abort_flag;
-  const bool copier = warp == kTqConsumers / 32;
-
-  // ---- copy the whole range in (the host sized it to fit the 4 stages)
-  if (copier && lane == 0) {
-    const uint8_t* src = static_cast<const uint8_t*>(args.in.x) + size_t(b_lo) * kBlockBytes;
-    for (uint32_t k = 0; k < n_stages; ++k) {
-      const uint32_t bytes = min(kStageBlocks, b_hi - b_lo - k * kStageBlocks) * kBlockBytes;
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_full + 8 * k),
-                   "r"(bytes)
-                   : "memory");
-      asm volatile(
-          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-              "r"(sbase + k * kTqStageBytes),
-          "l"(src + size_t(k) * kTqStageBytes), "r"(bytes), "r"(bar_full + 8 * k)
-          : "memory");
-    }
-  }
-  // ---- the range's amax
-  uint32_t mx = 0;
-  if (!copier) {
-    for (uint32_t k = 0; k < n_stages; ++k) {
-      if (!__all_sync(0xFFFFFFFFu,
-                      mbar_wait(bar_full + 8 * k, 0, ta.wait_limit_ns, abort, status)))
-        break;
-      const uint32_t n = min(kStageBlocks, b_hi - b_lo - k * kStageBlocks);
-      for (uint32_t i = threadIdx.x; i < n; i += kTqConsumers) {
-        RawBlock<InT> raw;
-        const uint32_t a = sbase + k * kTqStageBytes + i * kBlockBytes;
-#pragma unroll
-        for (uint32_t v = 0; v < kBlockBytes / 16; ++v) {
-          uint32_t* w = reinterpret_cast<uint32_t*>(&raw) + 4 * v;
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                       : "r"(a + 16 * v));
-        }
-        mx = max(mx, max(unit_absmax<InT>(raw.h[0]), unit_absmax<InT>(raw.h[1])));
-      }
-    }
-    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (lane == 0) warp_max[warp] = mx;
-  }
-  __syncthreads();
-  // ---- grid barrier: every CTA has raised the amax word
-  if (threadIdx.x == 0) {
-    uint32_t v = 0;
-    for (int w = 0; w < kTqConsumers / 32; ++w) v = max(v, warp_max[w]);
-    if (v != 0) atomicMax(amax_word, v);
-    uint32_t seen;
-    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], 1;" : "=r"(seen) : "l"(arrive) : "memory");
-    const uint64_t t0 = gtimer();
-    while (true) {
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(arrive) : "memory");
-      if (seen >= gridDim.x) break;
-      if (*abort || gtimer() - t0 > ta.wait_limit_ns) {
-        record_status(status, NVFP4_ERR_TIMEOUT);
-        *abort = 1;
-        break;
-      }
-    }
-    uint32_t bits;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(bits) : "l"(amax_word) : "memory");
-    s_t_shared = __fdiv_rn(__uint_as_float(bits), 2688.0f);
-  }
-  __syncthreads();
-  const float s_t = s_t_shared;
-  const bool in_domain = tensor_scale_in_domain(s_t);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    *args.s_t_out = s_t;
-    if (!in_domain) record_status(status, NVFP4_ERR_DOMAIN);
-  }
-  // ---- code the range out of shared memory
-  if (!copier && in_domain && !*abort) {
-    const ScaleConsts kc = make_consts(s_t);
-    for (uint32_t k = 0; k < n_stages; ++k) {
-      const uint32_t base = b_lo + k * kStageBlocks;
-      const uint32_t n = min(kStageBlocks, b_hi - base);
-      for (uint32_t i = threadIdx.x; i < n; i += kTqConsumers) {
-        RawBlock<InT> raw;
-        const uint32_t a = sbase + k * kTqStageBytes + i * kBlockBytes;
-#pragma unroll
-        for (uint32_t v = 0; v < kBlockBytes / 16; ++v) {
-          uint32_t* w = reinterpret_cast<uint32_t*>(&raw) + 4 * v;
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                       : "r"(a + 16 * v));
-        }
-        uint2 codes;
-        const uint32_t sb = quantize_block<InT>(raw, inv_tab, kc, codes);
-        const uint32_t b = base + i;
-        reinterpret_cast<uint2*>(args.codes)[b] = codes;
-        if (kSfLayout == NVFP4_SF_ROWMAJOR) {
-          args.sf[b] = uint8_t(sb);
-        } else {
-          const uint32_t row = fast_div(args.nkb_div, b);
-          args.sf[sf_mma_offset(row, b - row * args.nkb, args.ktiles)] = uint8_t(sb);
-        }
-      }
-    }
-  }
-  if (kSfLayout == NVFP4_SF_MMA128x4 && !copier) {
-    const uint32_t nkb4 = args.ktiles * 4u;
-    const uint32_t pad_rows = (args.rows_pad - args.rows) * nkb4;
-    const uint32_t pad_cols = args.rows * (nkb4 - args.nkb);
-    for (uint32_t i = blockIdx.x * kTqConsumers + threadIdx.x; i < pad_rows + pad_cols;
-         i += gridDim.x * kTqConsumers) {
-      uint32_t row, kb;
-      if (i < pad_rows) {
-        row = args.rows + i / nkb4;
-        kb = i % nkb4;
-      } else {
-        uint32_t j = i - pad_rows, extra = nkb4 - args.nkb;
-        row = j / extra;
-        kb = args.nkb + j % extra;
-      }
-      args.sf[sf_mma_offset(row, kb, args.ktiles)] = 0;
-    }
-  }
-  // ---- every copy landed before the CTA leaves (they did unless a wait ran out)
-  if (copier && lane == 0) {
-    for (uint32_t k = 0; k < n_stages; ++k) {
-      const uint64_t t0 = gtimer();
-      while (!mbar_try_wait(bar_full + 8 * k, 0)) {
-        if (gtimer() - t0 > 2000000000ull) {
-          record_status(status, NVFP4_ERR_TIMEOUT);
-          break;
-        }
-      }
-    }
-  }
-  // ---- leave: the last CTA out resets the barrier and the amax word
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t done;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(done) : "l"(depart) : "memory");
-    if (done == gridDim.x - 1) {
-      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(amax_word) : "memory");
-      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(arrive) : "memory");
-      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(depart) : "memory");
-    }
-  }
-}
-
 // ---- KV chunks staged through shared memory (K and V planes: blockIdx.y)
 // The chunk's tokens are rows of heads * head_dim contiguous elements at
 // token_stride apart (a fused QKV output, or a plain [tokens][heads][dim]
@@ -1255,77 +1072,10 @@ static cudaError_t launch_kv_encode_tma(KvTmaArgs ta, int sm_count, cudaStream_t
                     st, ta);
 }
 
-// The one-pass quantizer, when the tensor fits the rings of one resident
-// wave; returns cudaErrorNotSupported (nothing launched) when it does not.
-template <typename InT, int kSfLayout>
-static cudaError_t launch_fused(const QuantArgs& a, int sm_count, uint64_t wait_limit_ns,
-                                cudaStream_t st) {
-  static std::atomic<int> per_sm_cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  int per_sm = per_sm_cache[dev].load(std::memory_order_acquire);
-  if (per_sm == 0) {
-    cudaError_t e = cudaFuncSetAttribute(quant_fused_kernel<InT, kSfLayout>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kTqSmem);
-    if (e != cudaSuccess) return e;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_fused_kernel<InT, kSfLayout>,
-                                                      kTqThreads, kTqSmem) != cudaSuccess ||
-        per_sm < 1)
-      per_sm = 1;
-    per_sm_cache[dev].store(per_sm, std::memory_order_release);
-  }
-  constexpr uint32_t kStageBlocks = kTqStageBytes / (16 * sizeof(InT));
-  const uint32_t blocks = a.in.units >> 1;
-  uint32_t grid = (blocks + kStageBlocks - 1) / kStageBlocks;
-  const uint32_t cap = uint32_t(per_sm) * uint32_t(sm_count);
-  if (grid > cap) grid = cap;
-  if (grid < 1) grid = 1;
-  const uint32_t per_cta = (blocks + grid - 1) / grid;
-  if (per_cta > uint32_t(kTqStages) * kStageBlocks) return cudaErrorNotSupported;
-  TmaQuantArgs ta;
-  ta.q = a;
-  ta.per_cta = per_cta;
-  ta.wait_limit_ns = wait_limit_ns;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kTqThreads);
-  cfg.dynamicSmemBytes = size_t(kTqSmem);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeCooperative;
-  attr[1].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, quant_fused_kernel<InT, kSfLayout>, ta);
-}
-
 template <typename InT>
 static cudaError_t launch_quant_t(const LaunchQuant& q, cudaStream_t st) {
   const bool contig = (q.ld == q.cols);
   InMap m = make_inmap(q.x, q.rows, q.cols, 1, q.ld, 0);
-  if (!q.s_t_in && !q.amax_in && contig) {
-    // amax and codes in one pass over HBM when the tensor fits on chip
-    QuantArgs a;
-    a.in = m;
-    a.codes = q.codes;
-    a.sf = q.sf;
-    a.s_t_out = q.s_t_out;
-    a.s_t_in = nullptr;
-    a.amax_in = nullptr;
-    a.ws = static_cast<uint32_t*>(q.ws);
-    a.nkb = uint32_t(q.cols / 16);
-    a.nkb_div = make_fastdiv(a.nkb);
-    a.ktiles = (a.nkb + 3) / 4;
-    a.rows = uint32_t(q.rows);
-    a.rows_pad = uint32_t((q.rows + 127) / 128 * 128);
-    const bool mma = q.sf_layout == NVFP4_SF_MMA128x4;
-    const cudaError_t e =
-        mma ? launch_fused<InT, NVFP4_SF_MMA128x4>(a, q.sm_count, q.wait_limit_ns, st)
-            : launch_fused<InT, NVFP4_SF_ROWMAJOR>(a, q.sm_count, q.wait_limit_ns, st);
-    if (e != cudaErrorNotSupported) return e;
-  }
   if (!q.s_t_in && !q.amax_in) {
     AmaxArgs aa;
     aa.in[0] = m;
