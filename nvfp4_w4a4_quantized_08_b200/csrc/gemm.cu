@@ -762,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace gemm
 
 // ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -779,7 +779,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // 2-D map over uint8 code rows: box of 128 bytes x box_rows, 128-byte swizzle.
 static bool make_code_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
                           uint32_t box_rows) {
-  auto encode = get_encode();
+  auto encode = tensor_map_encoder();
   if (!encode) return false;
   cuuint64_t dims[2] = {row_bytes, rows};
   cuuint64_t strides[1] = {row_bytes};
@@ -796,7 +796,7 @@ static bool make_code_map(CUtensorMap* map, const void* base, uint64_t row_bytes
 // 128 bytes x 32 rows, 128-byte swizzle (the epilogue's staging layout).
 static bool make_out_map(CUtensorMap* map, void* base, int32_t dtype, uint64_t rows, uint64_t cols,
                          uint64_t ldc) {
-  auto encode = get_encode();
+  auto encode = tensor_map_encoder();
   if (!encode) return false;
   const uint64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
   cuuint64_t dims[2] = {cols, rows};

@@ -2,12 +2,18 @@
 // kernel files.  Arguments arrive here already validated.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "../../include/nvfp4.h"
 
 namespace nvfp4 {
+
+// cuTensorMapEncodeTiled from the driver, looked up once per process (null
+// when the driver does not provide it).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 struct LaunchQuant {
   const void* x;

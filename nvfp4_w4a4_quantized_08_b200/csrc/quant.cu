@@ -9,18 +9,23 @@
 // "Entrenamiento NVFP4").  KV chunks of up to 8 frames share one tensor scale
 // (hyper.ai LongLive-2.0 summary, section "方法").
 //
-// Exactness without a division per element.  Both roundings above are
-// monotone, so a value's code is pinned once two products that bracket the
-// correctly rounded quotient give the same code.  With r = RN(1/c) (c = 6 s_t)
-// and p = RN(RN(1/s_t) * RN(1/s_b)), the products RN(a * RN(r (1 -+ 2^-20)))
-// and RN(|x| * RN(p (1 -+ 2^-20))) lie below / above RN(a / c) and
-// RN(|x| / RN(s_b s_t)): each carries at most six roundings of relative size
-// 2^-24, far inside the 2^-20 margin.  Where the two codes differ (the quotient
-// sits within ~2^-20 of an E4M3 or E2M1 rounding boundary, a few times in a
-// million elements) the kernel takes the IEEE quotient itself.  Denormal
-// products only arise for values far below the smallest decision point, where
-// both bracket ends already give code 0.
+// Exact quotients without a division per element.  Every quotient of the
+// recipe is x / d with d fixed for a tensor (d = RN(6 s_t)) or a block
+// (d = RN(s_b s_t)); the kernels hold, per d, y = RN(1/d), y_rd = RD(1/d) and
+// y_lo = RN((1 - d y_rd) y_rd), form q0 = RN(x y_rd + RN(x y_lo)), within one
+// ulp of x / d, and correct it once with the exact remainder:
+// q = RN(q0 + (x - d q0) y) = RN(x / d) (Markstein's theorem: a faithful
+// quotient corrected with the correctly rounded reciprocal gives the correctly
+// rounded quotient).  Quotients below 2^-10 may lose their last bits (the
+// theorem assumes no underflow) but keep their sign and code to zero either
+// way.  Exact ties on E2M1 or E4M3 rounding boundaries, frequent when the
+// tensor scale has a short significand (an amax whose significand is a
+// multiple of 21 makes s_t = amax / 2688 exact), need no special path.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -177,113 +182,83 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(AmaxArgs args) {
 }
 
 // ---------------------------------------------------------------- encode pass
+// Division entry of a divisor d (see the file header).  The reciprocals are
+// stored negated and the kernels divide -x: with the operands in this order a
+// zero quotient keeps the dividend's sign, as IEEE division does (round to
+// nearest adds opposite zeros to +0; here only zeros of one sign meet).
+// y_lo >= 0 because y_rd <= 1/d.
+struct DivEnt {
+  float d, ny_rd, ny_lo, ny_rn;
+};
+
+__device__ __forceinline__ DivEnt div_entry(float d) {
+  const float y_rd = __frcp_rd(d);
+  const float rho = __fmaf_rn(-d, y_rd, 1.0f);  // 1 - d y_rd, exact
+  DivEnt e;
+  e.d = d;
+  e.ny_rd = -y_rd;
+  e.ny_lo = -__fmul_rn(rho, y_rd);
+  e.ny_rn = -__frcp_rn(d);
+  return e;
+}
+
+// RN(x / d), given nx = -x.
+__device__ __forceinline__ float div_rn(const DivEnt& e, float nx) {
+  const float q0 = __fmaf_rn(nx, e.ny_rd, __fmul_rn(nx, e.ny_lo));
+  const float r = __fmaf_rn(e.d, q0, nx);  // d q0 - x, exact
+  return __fmaf_rn(r, e.ny_rn, q0);
+}
+
+// The same for two dividends on the packed fp32 pipe.
+__device__ __forceinline__ float2 div_rn2(const DivEnt& e, float2 nx) {
+  const float2 q0 = __ffma2_rn(nx, make_float2(e.ny_rd, e.ny_rd),
+                               __fmul2_rn(nx, make_float2(e.ny_lo, e.ny_lo)));
+  const float2 r = __ffma2_rn(make_float2(e.d, e.d), q0, nx);
+  return __ffma2_rn(r, make_float2(e.ny_rn, e.ny_rn), q0);
+}
+
 struct ScaleConsts {
-  float s_t, c, rc_lo, rc_hi, inv_st;
+  DivEnt c;  // divisor of the block scale: RN(top * s_t)
+  float s_t;
   bool zero;
 };
 
-// Constants of the block-scale division amax_b / (top * s_t); top = 6 is the
+// Constants of the block-scale quotient amax_b / (top * s_t); top = 6 is the
 // recipe, 4 the Four Over Six alternative.
 __device__ __forceinline__ ScaleConsts make_consts(float s_t, float top = 6.0f) {
   ScaleConsts k;
   k.s_t = s_t;
   k.zero = (s_t == 0.0f);
-  k.c = __fmul_rn(top, s_t);
-  float rc = k.zero ? 0.0f : __frcp_rn(k.c);
-  k.rc_lo = __fmul_rn(rc, 1.0f - 0x1p-20f);
-  k.rc_hi = __fmul_rn(rc, 1.0f + 0x1p-20f);
-  k.inv_st = k.zero ? 0.0f : __frcp_rn(s_t);
+  k.c = div_entry(__fmul_rn(top, s_t));
   return k;
 }
 
-// The exact fallbacks below are out of line on purpose: inlined, the compiler
-// predicates them into the common path, which then issues their divisions for
-// every block.  A call is always a real branch.  They are not rare enough to
-// ignore: bf16 inputs and a tensor scale derived from a bf16 amax put 0.1 to
-// 1 percent of quotients exactly on (or within 2^-20 of) a rounding boundary,
-// so a few percent of blocks, and most warps, meet one.
-__device__ __noinline__ uint32_t e4m3_of_quotient(float a, float c) {
-  return e4m3x2(0.0f, __fdiv_rn(a, c)) & 0xFFu;
+// Division entries of d = RN(s_b s_t) for every scale byte (entry 0 and the
+// NaN byte 0x7F are never used for codes), one CTA's copy in shared memory.
+__device__ __forceinline__ void fill_div_table(DivEnt* tab, float s_t, uint32_t tid,
+                                               uint32_t nthreads) {
+  for (uint32_t b = tid; b < 128; b += nthreads)
+    tab[b] = div_entry(__fmul_rn(e4m3_to_f32(b), s_t));
 }
 
-__device__ __noinline__ uint32_t e2m1_of_quotient(float a, float d) {
-  const float y = __fdiv_rn(a, d);
-  return e2m1x8(y, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f) & 0xFu;
-}
-
-// E4M3 block scale of a block with amax amax_b: E4M3_RNE_sat(amax_b / c).
-__device__ __forceinline__ uint32_t block_scale(float amax_b, const ScaleConsts& k) {
-  uint32_t two = e4m3x2(__fmul_rn(amax_b, k.rc_hi), __fmul_rn(amax_b, k.rc_lo));
-  uint32_t sb = two & 0xFFu;
-  if (sb != (two >> 8)) sb = e4m3_of_quotient(amax_b, k.c);
-  return k.zero ? 0u : sb;
-}
-
-// E2M1 codes of the 16 elements of a block (x in a) for block scale byte sb,
-// from the two bracketing products: lo/hi code words of each half.  The codes
-// carry the sign (E2M1 is sign-magnitude and rounding to nearest even is
-// symmetric, so code(-y) = 8 | code(y); a negative value that rounds to zero
-// gives -0).  Nibbles where lo and hi differ need the exact quotient.
-__device__ __forceinline__ void bracket_codes(const float a[16], float inv_sb,
-                                              const ScaleConsts& k, uint32_t lo[2],
-                                              uint32_t hi[2]) {
-  const float p = __fmul_rn(k.inv_st, inv_sb);
-  const float p_lo = __fmul_rn(p, 1.0f - 0x1p-20f);
-  const float p_hi = __fmul_rn(p, 1.0f + 0x1p-20f);
-  // products on the packed fp32 pipe, two elements per instruction
-  float l[16], h[16];
-  const float2 plo2 = make_float2(p_lo, p_lo), phi2 = make_float2(p_hi, p_hi);
-#pragma unroll
-  for (int i = 0; i < 16; i += 2) {
-    const float2 ai = make_float2(a[i], a[i + 1]);
-    const float2 vl = __fmul2_rn(ai, plo2), vh = __fmul2_rn(ai, phi2);
-    l[i] = vl.x; l[i + 1] = vl.y;
-    h[i] = vh.x; h[i + 1] = vh.y;
-  }
-  lo[0] = e2m1x8(l[0], l[1], l[2], l[3], l[4], l[5], l[6], l[7]);
-  lo[1] = e2m1x8(l[8], l[9], l[10], l[11], l[12], l[13], l[14], l[15]);
-  hi[0] = e2m1x8(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]);
-  hi[1] = e2m1x8(h[8], h[9], h[10], h[11], h[12], h[13], h[14], h[15]);
-}
-
-// Element i (0..7) of a unit as binary32, selected without indexing the
-// register array dynamically (which would move it to local memory).
+// The 8 elements of a unit negated, as binary32 (flipping the sign bits
+// first; bf16 -> binary32 is exact).
 template <typename InT>
-__device__ __forceinline__ float elem_value(const Raw<InT>& r, uint32_t i);
+__device__ __forceinline__ void unit_neg_values(const Raw<InT>& r, float a[8]);
 template <>
-__device__ __forceinline__ float elem_value<__nv_bfloat16>(const Raw<__nv_bfloat16>& r,
-                                                           uint32_t i) {
-  const uint32_t j = i >> 1;
-  uint32_t w = r.w[0];
-  w = j == 1 ? r.w[1] : w;
-  w = j == 2 ? r.w[2] : w;
-  w = j == 3 ? r.w[3] : w;
-  return __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+__device__ __forceinline__ void unit_neg_values<__nv_bfloat16>(const Raw<__nv_bfloat16>& r,
+                                                               float a[8]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w = r.w[j] ^ 0x80008000u;
+    a[2 * j] = __uint_as_float(w << 16);
+    a[2 * j + 1] = __uint_as_float(w & 0xFFFF0000u);
+  }
 }
 template <>
-__device__ __forceinline__ float elem_value<float>(const Raw<float>& r, uint32_t i) {
-  uint32_t w = r.w[0];
+__device__ __forceinline__ void unit_neg_values<float>(const Raw<float>& r, float a[8]) {
 #pragma unroll
-  for (uint32_t j = 1; j < 8; ++j) w = i == j ? r.w[j] : w;
-  return __uint_as_float(w);
-}
-
-// Replace the codes of a unit whose two bracket codes differ (nonzero nibbles
-// of diff) by the codes of the IEEE quotients x / d, d = RN(s_b s_t).
-template <typename InT>
-__device__ __forceinline__ uint32_t patch_codes(const Raw<InT>& r, uint32_t c, uint32_t diff,
-                                                float d) {
-  while (diff) {
-    const uint32_t sh = (__ffs(diff) - 1) & ~3u;
-    c = (c & ~(0xFu << sh)) | (e2m1_of_quotient(elem_value<InT>(r, sh >> 2), d) << sh);
-    diff &= ~(0xFu << sh);
-  }
-  return c;
-}
-
-__device__ __forceinline__ void fill_inv_table(float* tab) {
-  for (int b = threadIdx.x; b < 128; b += blockDim.x)
-    tab[b] = (b == 0 || b == 0x7F) ? 0.0f : __frcp_rn(e4m3_to_f32(b));
+  for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(r.w[i] ^ 0x80000000u);
 }
 
 // The plane's tensor scale: s_t_in if given, else amax / 2688 with the amax
@@ -352,26 +327,28 @@ __device__ __forceinline__ uint32_t sf_mma_offset(uint32_t row, uint32_t kb, uin
 }
 
 // Quantize one block held in `raw`: returns its scale byte and writes its two
-// code words (all +0 when the scale is 0).
+// code words (all +0 when the scale is 0).  E2M1 is sign-magnitude and round
+// to nearest even is symmetric, so the sign of x carries into the code, and a
+// negative value that rounds to zero gives -0.
 template <typename InT>
-__device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, const float* inv_tab,
+__device__ __forceinline__ uint32_t quantize_block(const RawBlock<InT>& raw, const DivEnt* tab,
                                                    const ScaleConsts& k, uint2& codes) {
-  uint32_t sb, lo[2], hi[2];
-  {
-    const uint32_t mx = max(unit_absmax<InT>(raw.h[0]), unit_absmax<InT>(raw.h[1]));
-    sb = block_scale(__uint_as_float(mx), k);
-    float a[16];
-    unit_values<InT>(raw.h[0], a);
-    unit_values<InT>(raw.h[1], a + 8);
-    bracket_codes(a, inv_tab[sb & 0x7Fu], k, lo, hi);
+  const uint32_t mx = max(unit_absmax<InT>(raw.h[0]), unit_absmax<InT>(raw.h[1]));
+  const uint32_t sb =
+      k.zero ? 0u : (e4m3x2(0.0f, div_rn(k.c, -__uint_as_float(mx))) & 0xFFu);
+  const DivEnt e = tab[sb & 0x7Fu];
+  float na[16], q[16];
+  unit_neg_values<InT>(raw.h[0], na);
+  unit_neg_values<InT>(raw.h[1], na + 8);
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const float2 v = div_rn2(e, make_float2(na[i], na[i + 1]));
+    q[i] = v.x;
+    q[i + 1] = v.y;
   }
-  const uint32_t diff0 = lo[0] ^ hi[0], diff1 = lo[1] ^ hi[1];
-  if (diff0 | diff1) {
-    const float d = __fmul_rn(e4m3_to_f32(sb), k.s_t);
-    lo[0] = patch_codes<InT>(raw.h[0], lo[0], diff0, d);
-    lo[1] = patch_codes<InT>(raw.h[1], lo[1], diff1, d);
-  }
-  codes = sb ? make_uint2(lo[0], lo[1]) : make_uint2(0u, 0u);
+  codes = sb ? make_uint2(e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]),
+                          e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]))
+             : make_uint2(0u, 0u);
   return sb;
 }
 
@@ -440,12 +417,12 @@ __device__ __noinline__ bool four_beats_six_exact(const RawBlock<InT> raw, uint2
 // order is certainly the binary64 one; otherwise in binary64.
 template <typename InT>
 __device__ __forceinline__ uint32_t quantize_block_4over6(const RawBlock<InT>& raw,
-                                                          const float* inv_tab,
+                                                          const DivEnt* tab,
                                                           const ScaleConsts& k6,
                                                           const ScaleConsts& k4, uint2& codes) {
   uint2 c6, c4;
-  const uint32_t sb6 = quantize_block<InT>(raw, inv_tab, k6, c6);
-  const uint32_t sb4 = quantize_block<InT>(raw, inv_tab, k4, c4);
+  const uint32_t sb6 = quantize_block<InT>(raw, tab, k6, c6);
+  const uint32_t sb4 = quantize_block<InT>(raw, tab, k4, c4);
   codes = c6;
   if (sb4 == sb6) return sb6;
   float a[16];
@@ -472,9 +449,7 @@ __device__ __forceinline__ uint32_t quantize_block_4over6(const RawBlock<InT>& r
 template <typename InT, bool kContig, int kSfLayout>
 __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args) {
   constexpr int D = Prefetch<InT>::kDepth;
-  __shared__ float inv_tab[128];
-  fill_inv_table(inv_tab);
-  __syncthreads();
+  __shared__ DivEnt div_tab[128];
   pdl_wait();
   pdl_trigger();
   const uint32_t stride = gridDim.x * blockDim.x;
@@ -492,6 +467,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args)
     *args.s_t_out = s_t;
     if (!in_domain) record_status(args.ws + kWsStatus / 4, NVFP4_ERR_DOMAIN);
   }
+  fill_div_table(div_tab, s_t, threadIdx.x, blockDim.x);
+  __syncthreads();
   if (in_domain) {
     const ScaleConsts k = make_consts(s_t);
     for (; b0 < blocks; b0 += D * stride) {
@@ -506,7 +483,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_kernel(QuantArgs args)
         const uint32_t b = b0 + i * stride;
         if (b < blocks) {
           uint2 codes;
-          const uint32_t sb = quantize_block<InT>(cur[i], inv_tab, k, codes);
+          const uint32_t sb = quantize_block<InT>(cur[i], div_tab, k, codes);
           reinterpret_cast<uint2*>(args.codes)[b] = codes;
           if (kSfLayout == NVFP4_SF_ROWMAJOR) {
             args.sf[b] = uint8_t(sb);
@@ -604,13 +581,12 @@ __global__ void __launch_bounds__(kTqThreads) quant_tma_kernel(const TmaQuantArg
   constexpr uint32_t kStageBlocks = kTqStageBytes / kBlockBytes;
   const QuantArgs& args = ta.q;
   extern __shared__ __align__(128) uint8_t tq_smem[];
-  __shared__ float inv_tab[128];
+  __shared__ DivEnt div_tab[128];
   __shared__ int abort_flag;
   const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(tq_smem));
   const uint32_t bar_full = sbase + kTqStages * kTqStageBytes;
   const uint32_t bar_empty = bar_full + 8 * kTqStages;
   uint32_t* const status = args.ws + kWsStatus / 4;
-  fill_inv_table(inv_tab);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTqStages; ++s) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_full + 8 * s) : "memory");
@@ -673,6 +649,8 @@ __global__ void __launch_bounds__(kTqThreads) quant_tma_kernel(const TmaQuantArg
       *args.s_t_out = s_t;
       if (!in_domain) record_status(status, NVFP4_ERR_DOMAIN);
     }
+    fill_div_table(div_tab, s_t, threadIdx.x, kTqConsumers);
+    asm volatile("bar.sync 1, %0;" ::"n"(kTqConsumers) : "memory");  // encoders only
     const ScaleConsts kc = make_consts(s_t);
     for (uint32_t k = 0; k < n_stages; ++k) {
       const uint32_t s = k % kTqStages;
@@ -696,7 +674,7 @@ __global__ void __launch_bounds__(kTqThreads) quant_tma_kernel(const TmaQuantArg
                            : "r"(a + 16 * v));
             }
             uint2 codes;
-            const uint32_t sb = quantize_block<InT>(raw, inv_tab, kc, codes);
+            const uint32_t sb = quantize_block<InT>(raw, div_tab, kc, codes);
             const uint32_t b = base + i;
             reinterpret_cast<uint2*>(args.codes)[b] = codes;
             if (kSfLayout == NVFP4_SF_ROWMAJOR) {
@@ -736,6 +714,239 @@ __global__ void __launch_bounds__(kTqThreads) quant_tma_kernel(const TmaQuantArg
   check_in(args.s_t_in, args.amax_in, args.ws, 0);
 }
 
+// ---- bf16 tensors whose rows are a multiple of 64 elements, tile by tile
+// The tensor is cut into tiles of 128 rows x 64 columns: 16 KB of bf16, whose
+// 128 x 4 scale bytes are exactly one 512-byte tile of the tensor-core scale
+// layout.  A resident grid of CTAs takes equal runs of tiles (row-major tile
+// order).  Warp 8 (one lane) loads each tile with one 2-D TMA copy (128-byte
+// swizzle) into a 4-stage ring; warps 0..7 encode it.  Thread t takes row
+// t / 2 and blocks 2 (t % 2), 2 (t % 2) + 1 of the tile (64 bytes of its row):
+// its four 16-byte chunks sit at swizzled positions that differ across the 8
+// threads of a quarter warp, so the shared-memory reads have no bank
+// conflicts; the warp releases the stage once the chunks are in registers.
+// The thread stores its 16 bytes of codes (the two threads of a row fill a
+// 32-byte sector together) and its two scale bytes.  Rows past the end of the
+// tensor arrive as zeros from the TMA copy: their scale bytes are the zero
+// padding the tensor-core layout needs, and their codes are not stored.
+constexpr int kTtConsumers = 256;
+constexpr int kTtThreads = kTtConsumers + 32;
+constexpr int kTtRows = 128;
+constexpr int kTtStageBytes = kTtRows * 128;
+constexpr int kTtStages = 4;
+// ring (1024-byte aligned: the swizzle pattern repeats every 8 rows of 128 B),
+// the barriers, and the alignment slack
+constexpr int kTtSmem = kTtStages * kTtStageBytes + 2 * kTtStages * 8 + 1024;
+
+struct TileQuantArgs {
+  QuantArgs q;
+  uint32_t n_ct;      // column tiles: cols / 64
+  uint32_t n_tiles;   // row tiles * column tiles
+  uint32_t per_cta;   // tiles per CTA (the first `extra` CTAs take one more)
+  uint32_t extra;
+  uint64_t wait_limit_ns;
+};
+
+// Division entry of a divisor with each value twice, for the packed fp32 pipe.
+struct DivEnt2 {
+  float2 d, ny_rd, ny_lo, ny_rn;
+};
+
+__device__ __forceinline__ float2 div_rn2(const DivEnt2& e, float2 nx) {
+  const float2 q0 = __ffma2_rn(nx, e.ny_rd, __fmul2_rn(nx, e.ny_lo));
+  const float2 r = __ffma2_rn(e.d, q0, nx);
+  return __ffma2_rn(r, e.ny_rn, q0);
+}
+
+__device__ __forceinline__ DivEnt2 div_entry2(float d) {
+  const DivEnt e = div_entry(d);
+  DivEnt2 e2;
+  e2.d = make_float2(e.d, e.d);
+  e2.ny_rd = make_float2(e.ny_rd, e.ny_rd);
+  e2.ny_lo = make_float2(e.ny_lo, e.ny_lo);
+  e2.ny_rn = make_float2(e.ny_rn, e.ny_rn);
+  return e2;
+}
+
+// max |x| over the 16 bf16 of a block (8 words), as binary32 bits: a tree of
+// packed magnitude maxima (their signs are the xor of the operands' and are
+// dropped at the end), then the larger half.
+__device__ __forceinline__ uint32_t bf16_block_absmax(const uint32_t w[8]) {
+  uint32_t m[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[i]) : "r"(w[2 * i]), "r"(w[2 * i + 1]));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[0]) : "r"(m[0]), "r"(m[1]));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[2]) : "r"(m[2]), "r"(m[3]));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[0]) : "r"(m[0]), "r"(m[2]));
+  const uint32_t a = m[0] & 0x7FFF7FFFu;
+  uint32_t b;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(b) : "r"(a), "r"(prmt(a, 0u, 0x1032u)));
+  return b << 16;
+}
+
+// Codes of one bf16 block (8 words) for a block with division entry e.
+__device__ __forceinline__ uint2 bf16_block_codes(const uint32_t w[8], const DivEnt2& e) {
+  float q[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    // -x of both halves: the low half moved up with its sign bit flipped
+    // (adding 2^31 flips bit 31), the high half masked and flipped
+    const float2 nx = make_float2(__uint_as_float(w[j] * 0x10000u + 0x80000000u),
+                                  __uint_as_float((w[j] & 0xFFFF0000u) ^ 0x80000000u));
+    const float2 v = div_rn2(e, nx);
+    q[2 * j] = v.x;
+    q[2 * j + 1] = v.y;
+  }
+  return make_uint2(e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]),
+                    e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]));
+}
+
+template <int kSfLayout>
+__global__ void __launch_bounds__(kTtThreads) quant_tile_kernel(
+    const __grid_constant__ CUtensorMap map_x, const TileQuantArgs ta) {
+  const QuantArgs& args = ta.q;
+  extern __shared__ uint8_t tt_smem[];
+  __shared__ DivEnt2 div_tab[128];
+  __shared__ int abort_flag;
+  const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(tt_smem));
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  const uint32_t bar_full = sbase + kTtStages * kTtStageBytes;
+  const uint32_t bar_empty = bar_full + 8 * kTtStages;
+  uint32_t* const status = args.ws + kWsStatus / 4;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTtStages; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_full + 8 * s) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar_empty + 8 * s),
+                   "r"(kTtConsumers / 32)
+                   : "memory");
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (threadIdx.x == kTtConsumers)
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&map_x) : "memory");
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t t_lo = blockIdx.x * ta.per_cta + min(blockIdx.x, ta.extra);
+  const uint32_t n_local = ta.per_cta + (blockIdx.x < ta.extra ? 1u : 0u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &abort_flag;
+
+  if (warp == kTtConsumers / 32) {
+    // ------------------------------------------------------------ TMA warp
+    if (lane == 0) {
+      uint32_t k = 0;
+      for (; k < n_local; ++k) {
+        const uint32_t s = k % kTtStages;
+        if (!mbar_wait(bar_empty + 8 * s, ((k / kTtStages) & 1) ^ 1, ta.wait_limit_ns, abort,
+                       status))
+          break;
+        const uint32_t tile = t_lo + k;
+        const uint32_t rt = tile / ta.n_ct, ct = tile - rt * ta.n_ct;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_full + 8 * s),
+                     "r"(kTtStageBytes)
+                     : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+            "[%0], [%1, {%2, %3}], [%4];" ::"r"(sbase + s * kTtStageBytes),
+            "l"(&map_x), "r"(int32_t(ct * 64)), "r"(int32_t(rt * kTtRows)), "r"(bar_full + 8 * s)
+            : "memory");
+      }
+      // drain: every copy issued has landed before the CTA may leave
+      for (uint32_t d = (k > kTtStages ? k - kTtStages : 0); d < k; ++d) {
+        const uint32_t s = d % kTtStages;
+        const uint64_t t0 = gtimer();
+        while (!mbar_try_wait(bar_full + 8 * s, (d / kTtStages) & 1)) {
+          if (gtimer() - t0 > 2000000000ull) {
+            record_status(status, NVFP4_ERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ encoders
+    const uint32_t tid = threadIdx.x;
+    const float s_t = read_scale(args.s_t_in, args.amax_in, args.ws, 0);
+    const bool in_domain = tensor_scale_in_domain(s_t);
+    if (blockIdx.x == 0 && tid == 0) {
+      *args.s_t_out = s_t;
+      if (!in_domain) record_status(status, NVFP4_ERR_DOMAIN);
+    }
+    if (tid < 128) div_tab[tid] = div_entry2(__fmul_rn(e4m3_to_f32(tid), s_t));
+    asm volatile("bar.sync 1, %0;" ::"n"(kTtConsumers) : "memory");  // encoders only
+    const DivEnt2 kc = div_entry2(__fmul_rn(6.0f, s_t));
+    const bool zero = s_t == 0.0f;
+    constexpr bool mma = kSfLayout == NVFP4_SF_MMA128x4;
+    const uint32_t r = tid >> 1, h = tid & 1;
+    // this thread's chunks (logical 4h .. 4h+3 of row r) in a stage
+    uint32_t off[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) off[j] = r * 128u + (((4u * h + j) ^ (r & 7u)) << 4);
+    const uint32_t sf_off = (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + 2u * h;
+    const size_t row_bytes = size_t(args.nkb) * 8u;
+    // the tile's row and column tile, advanced one tile per iteration
+    uint32_t rt = t_lo / ta.n_ct, ct = t_lo - rt * ta.n_ct;
+    for (uint32_t k = 0; k < n_local; ++k, ++ct) {
+      if (ct == ta.n_ct) {
+        ct = 0;
+        ++rt;
+      }
+      const uint32_t s = k % kTtStages;
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * s, (k / kTtStages) & 1,
+                                                        ta.wait_limit_ns, abort, status));
+      if (!ok) break;
+      uint32_t w[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[4 * j]), "=r"(w[4 * j + 1]), "=r"(w[4 * j + 2]), "=r"(w[4 * j + 3])
+                     : "r"(sbase + s * kTtStageBytes + off[j]));
+      // The stage is released after the stores below: a store cannot issue
+      // before the values it writes, and so the loads behind them, are
+      // complete.  Released straight after the loads, the next TMA copy into
+      // the stage could land before slow loads had read it (seen on B200 as
+      // a few corrupted blocks in large tensors).
+      auto release = [&]() {
+        __syncwarp();
+        if (lane == 0)
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_empty + 8 * s)
+                       : "memory");
+      };
+      if (!in_domain) {  // nothing is read from the stage
+        release();
+        continue;
+      }
+      const uint32_t am0 = bf16_block_absmax(w), am1 = bf16_block_absmax(w + 8);
+      // both block scales at once: amax_b / RN(6 s_t), then E4M3 (block 0 in
+      // the low byte)
+      const float2 qs = div_rn2(kc, make_float2(-__uint_as_float(am0), -__uint_as_float(am1)));
+      const uint32_t sb2 = zero ? 0u : e4m3x2(qs.y, qs.x);
+      const uint32_t sb0 = sb2 & 0xFFu, sb1 = sb2 >> 8;
+      uint2 c0 = bf16_block_codes(w, div_tab[sb0 & 0x7Fu]);
+      uint2 c1 = bf16_block_codes(w + 8, div_tab[sb1 & 0x7Fu]);
+      if (sb0 == 0) c0 = make_uint2(0u, 0u);
+      if (sb1 == 0) c1 = make_uint2(0u, 0u);
+      const uint32_t grow = rt * kTtRows + r;
+      if (grow < args.rows) {
+        st_v4(args.codes + size_t(grow) * row_bytes + ct * 32u + h * 16u,
+              make_uint4(c0.x, c0.y, c1.x, c1.y));
+        if (!mma)
+          *reinterpret_cast<uint16_t*>(args.sf + size_t(grow) * args.nkb + ct * 4u + 2u * h) =
+              uint16_t(sb2);
+      }
+      // tensor-core layout: tile (rt, ct) is scale tile rt * ktiles + ct =
+      // t_lo + k (ktiles == n_ct), padding rows included
+      if (mma)
+        *reinterpret_cast<uint16_t*>(args.sf + size_t(t_lo + k) * 512u + sf_off) = uint16_t(sb2);
+      release();
+    }
+  }
+  check_in(args.s_t_in, args.amax_in, args.ws, 0);
+}
+
 // ---- KV-cache chunks (K and V planes in one launch, blockIdx.y)
 struct KvQuantArgs {
   InMap in[2];
@@ -754,9 +965,7 @@ template <bool kContig, int kRule>
 __global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4 : 3)
     kv_quant_kernel(KvQuantArgs args) {
   constexpr int D = Prefetch<__nv_bfloat16>::kDepth;
-  __shared__ float inv_tab[128];
-  fill_inv_table(inv_tab);
-  __syncthreads();
+  __shared__ DivEnt div_tab[128];
   pdl_wait();
   pdl_trigger();
   const int plane = blockIdx.y;
@@ -778,6 +987,8 @@ __global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4
     args.st[plane][args.slots[threadIdx.x]] = s_t;
   if (blockIdx.x == 0 && threadIdx.x == 0 && !in_domain)
     record_status(args.ws + kWsStatus / 4, NVFP4_ERR_DOMAIN);
+  fill_div_table(div_tab, s_t, threadIdx.x, blockDim.x);
+  __syncthreads();
   if (in_domain) {
     uint8_t* const codes_pool = plane == 0 ? args.codes[0] : args.codes[1];
     uint8_t* const sf_pool = plane == 0 ? args.sf[0] : args.sf[1];
@@ -799,8 +1010,8 @@ __global__ void __launch_bounds__(kQuantThreads, kRule == NVFP4_SCALE_ONTO_6 ? 4
           uint2 codes;
           const uint32_t sb =
               kRule == NVFP4_SCALE_ONTO_6
-                  ? quantize_block<__nv_bfloat16>(cur[i], inv_tab, k, codes)
-                  : quantize_block_4over6<__nv_bfloat16>(cur[i], inv_tab, k, k4, codes);
+                  ? quantize_block<__nv_bfloat16>(cur[i], div_tab, k, codes)
+                  : quantize_block_4over6<__nv_bfloat16>(cur[i], div_tab, k, k4, codes);
           const uint32_t f = fast_div(args.bpf_div, b);
           const uint32_t bf = b - f * bpf;
           const size_t slot = size_t(args.slots[f]);
@@ -838,13 +1049,12 @@ template <int kRule>
 __global__ void __launch_bounds__(kTqThreads) kv_quant_tma_kernel(const KvTmaArgs ta) {
   const KvQuantArgs& args = ta.kv;
   extern __shared__ __align__(128) uint8_t kq_smem[];
-  __shared__ float inv_tab[128];
+  __shared__ DivEnt div_tab[128];
   __shared__ int abort_flag;
   const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(kq_smem));
   const uint32_t bar_full = sbase + kTqStages * kKvStageBytes;
   const uint32_t bar_empty = bar_full + 8 * kTqStages;
   uint32_t* const status = args.ws + kWsStatus / 4;
-  fill_inv_table(inv_tab);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTqStages; ++s) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_full + 8 * s) : "memory");
@@ -909,6 +1119,8 @@ __global__ void __launch_bounds__(kTqThreads) kv_quant_tma_kernel(const KvTmaArg
     if (blockIdx.x == 0 && threadIdx.x < args.n_frames)
       args.st[plane][args.slots[threadIdx.x]] = s_t;
     if (blockIdx.x == 0 && threadIdx.x == 0 && !in_domain) record_status(status, NVFP4_ERR_DOMAIN);
+    fill_div_table(div_tab, s_t, threadIdx.x, kTqConsumers);
+    asm volatile("bar.sync 1, %0;" ::"n"(kTqConsumers) : "memory");  // encoders only
     uint8_t* const codes_pool = plane == 0 ? args.codes[0] : args.codes[1];
     uint8_t* const sf_pool = plane == 0 ? args.sf[0] : args.sf[1];
     const ScaleConsts k6 = make_consts(s_t);
@@ -936,8 +1148,8 @@ __global__ void __launch_bounds__(kTqThreads) kv_quant_tma_kernel(const KvTmaArg
           uint2 codes;
           const uint32_t sb =
               kRule == NVFP4_SCALE_ONTO_6
-                  ? quantize_block<__nv_bfloat16>(raw, inv_tab, k6, codes)
-                  : quantize_block_4over6<__nv_bfloat16>(raw, inv_tab, k6, k4, codes);
+                  ? quantize_block<__nv_bfloat16>(raw, div_tab, k6, codes)
+                  : quantize_block_4over6<__nv_bfloat16>(raw, div_tab, k6, k4, codes);
           const uint32_t b = r0 * ta.row_blocks + i;   // block of the chunk
           const uint32_t f = fast_div(args.bpf_div, b);
           const uint32_t bf = b - f * bpf;
@@ -1045,6 +1257,57 @@ static cudaError_t launch_encode_tma(const QuantArgs& a, int sm_count, uint64_t 
                     size_t(kTqSmem), st, ta);
 }
 
+// 2-D map over a bf16 tensor [rows][cols] with contiguous rows: box of 64
+// columns (128 bytes) x 128 rows, 128-byte swizzle; rows past the end read as
+// zeros.
+static bool make_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, uint32_t(kTtRows)};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tile quantizer: one resident wave, the tiles split evenly over it.
+template <int kSfLayout>
+static cudaError_t launch_encode_tile(const QuantArgs& a, const void* x, uint64_t rows,
+                                      uint64_t cols, int sm_count, uint64_t wait_limit_ns,
+                                      cudaStream_t st) {
+  static std::atomic<int> per_sm_cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  int per_sm = per_sm_cache[dev].load(std::memory_order_acquire);
+  if (per_sm == 0) {
+    cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<kSfLayout>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kTtSmem);
+    if (e != cudaSuccess) return e;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tile_kernel<kSfLayout>,
+                                                      kTtThreads, kTtSmem) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    per_sm_cache[dev].store(per_sm, std::memory_order_release);
+  }
+  CUtensorMap map;
+  if (!make_bf16_tile_map(&map, x, rows, cols)) return cudaErrorInvalidValue;
+  TileQuantArgs ta;
+  ta.q = a;
+  ta.n_ct = uint32_t(cols / 64);
+  ta.n_tiles = uint32_t((rows + kTtRows - 1) / kTtRows) * ta.n_ct;
+  uint32_t grid = uint32_t(per_sm) * uint32_t(sm_count);
+  if (grid > ta.n_tiles) grid = ta.n_tiles;
+  if (grid < 1) grid = 1;
+  ta.per_cta = ta.n_tiles / grid;
+  ta.extra = ta.n_tiles % grid;
+  ta.wait_limit_ns = wait_limit_ns;
+  return launch_pdl(quant_tile_kernel<kSfLayout>, dim3(grid), dim3(kTtThreads), size_t(kTtSmem),
+                    st, map, ta);
+}
+
 template <int kRule>
 static cudaError_t launch_kv_encode_tma(KvTmaArgs ta, int sm_count, cudaStream_t st) {
   static std::atomic<int> per_sm_cache[64];
@@ -1099,7 +1362,15 @@ static cudaError_t launch_quant_t(const LaunchQuant& q, cudaStream_t st) {
   a.rows = uint32_t(q.rows);
   a.rows_pad = uint32_t((q.rows + 127) / 128 * 128);
   const bool mma = q.sf_layout == NVFP4_SF_MMA128x4;
-  // contiguous rows: the staged kernel (1-D bulk copies need 16-byte aligned
+  // bf16 rows of a multiple of 64 elements at a 16-byte aligned address: the
+  // tile kernel (2-D TMA copies)
+  if (std::is_same<InT, __nv_bfloat16>::value && contig && q.cols % 64 == 0 &&
+      reinterpret_cast<uintptr_t>(q.x) % 16 == 0)
+    return mma ? launch_encode_tile<NVFP4_SF_MMA128x4>(a, q.x, uint64_t(q.rows), uint64_t(q.cols),
+                                                       q.sm_count, q.wait_limit_ns, st)
+               : launch_encode_tile<NVFP4_SF_ROWMAJOR>(a, q.x, uint64_t(q.rows), uint64_t(q.cols),
+                                                       q.sm_count, q.wait_limit_ns, st);
+  // other contiguous rows: the staged kernel (1-D bulk copies need 16-byte aligned
   // addresses, which the C ABI's checks guarantee)
   if (contig)
     return mma ? launch_encode_tma<InT, NVFP4_SF_MMA128x4>(a, q.sm_count, q.wait_limit_ns, st)
