@@ -207,8 +207,22 @@ __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_wait_ld() {
+// Waits for every earlier tensor-memory load of the thread, then ties the
+// registers of both loads to the wait so that nothing reading them can be
+// scheduled before it.
+__device__ __forceinline__ void regs_after_wait(uint32_t (&r)[32]) {
+  asm volatile(
+      ""
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r0)[32], uint32_t (&r1)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  regs_after_wait(r0);
+  regs_after_wait(r1);
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -383,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
         uint32_t r0[32], r1[32];
         tmem_ld32_async(s_addr + 32 * c, r0);
         tmem_ld32_async(s_addr + 32 * c + 32, r1);
-        tmem_wait_ld();
+        tmem_wait_ld(r0, r1);
         if (!tail) {
 #pragma unroll
           for (uint32_t e = 0; e < 32; ++e)
@@ -414,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
         uint32_t r[2][32];
         tmem_ld32_async(s_addr + 32 * c, r[0]);
         tmem_ld32_async(s_addr + 32 * c + 32, r[1]);
-        tmem_wait_ld();
+        tmem_wait_ld(r[0], r[1]);
 #pragma unroll
         for (uint32_t h2 = 0; h2 < 2; ++h2) {
           uint32_t pk[16];

@@ -287,6 +287,36 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
   }
 }
 
+// The load without its wait; tmem_wait_ld32 waits for every earlier load of
+// the thread and then ties the registers of `r` to the wait, so that nothing
+// reading them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_regs_after_wait(uint32_t (&r)[32]) {
+  asm volatile(
+      ""
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+__device__ __forceinline__ void tmem_wait_ld2(uint32_t (&r0)[32], uint32_t (&r1)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  tmem_regs_after_wait(r0);
+  tmem_regs_after_wait(r1);
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -697,14 +727,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem + ((quad * 32) << 16) + half * 128;
       if (bf16) {
         uint32_t pk[64];
+        // two 32-column loads in flight per wait: the accumulator is released
+        // after two load latencies instead of four
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(taddr + 32 * c, r);
+        for (int c = 0; c < 4; c += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_async(taddr + 32 * c, r0);
+          tmem_ld32_async(taddr + 32 * c + 32, r1);
+          tmem_wait_ld2(r0, r1);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[16 * c + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+          for (int e = 0; e < 16; ++e) {
+            pk[16 * c + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r0[2 * e]), alpha),
+                                       __fmul_rn(__uint_as_float(r0[2 * e + 1]), alpha));
+            pk[16 * c + 16 + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r1[2 * e]), alpha),
+                                            __fmul_rn(__uint_as_float(r1[2 * e + 1]), alpha));
+          }
         }
         release();
         // the activation runs on the bf16 products once the accumulator is
