@@ -18,18 +18,20 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   return r;
 }
 
+// Only two products are rounded: f2 = RN(s_b s_t) and f3 = RN((1.5 s_b) s_t).
+// The other magnitudes are these times a power of two (0.5 f2, 2 f2, 2 f3,
+// 4 f2, 4 f3), and scaling by a power of two commutes with rounding to binary32
+// and to bf16 while nothing overflows or leaves the normal range, which the
+// tensor-scale domain guarantees (s_b s_t >= 2^-117, 6 s_b s_t < 2^112).  So
+// the bf16 words of 2 f and 4 f are those of f with 1 or 2 added to the
+// exponent field of each half, and of 0.5 f with 1 taken from it.  A zero
+// scale byte gives the all-zero table.
 __device__ __forceinline__ BlockLut make_lut(uint32_t sb, float s_t) {
   const float s = e4m3_to_f32(sb);
-  // (v * s_b) is exact; one rounding for * s_t, one for bf16
-  const float f1 = __fmul_rn(__fmul_rn(0.5f, s), s_t);
-  const float f2 = __fmul_rn(s, s_t);
-  const float f3 = __fmul_rn(__fmul_rn(1.5f, s), s_t);
-  const float f4 = __fmul_rn(__fmul_rn(2.0f, s), s_t);
-  const float f5 = __fmul_rn(__fmul_rn(3.0f, s), s_t);
-  const float f6 = __fmul_rn(__fmul_rn(4.0f, s), s_t);
-  const float f7 = __fmul_rn(__fmul_rn(6.0f, s), s_t);
-  const uint32_t t01 = bf16x2_rn(0.0f, f1), t23 = bf16x2_rn(f2, f3);
-  const uint32_t t45 = bf16x2_rn(f4, f5), t67 = bf16x2_rn(f6, f7);
+  const uint32_t t23 = bf16x2_rn(__fmul_rn(s, s_t), __fmul_rn(__fmul_rn(1.5f, s), s_t));
+  const uint32_t e1 = t23 ? 0x00800080u : 0u;  // +1 in both exponent fields
+  const uint32_t t45 = t23 + e1, t67 = t23 + 2 * e1;
+  const uint32_t t01 = (t23 - (e1 & 0xFFFFu)) << 16;  // (0, 0.5 f2)
   BlockLut l;
   l.lo0 = prmt(t01, t23, 0x6420);
   l.hi0 = prmt(t01, t23, 0x7531);
