@@ -210,6 +210,13 @@ __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32
 // Waits for every earlier tensor-memory load of the thread, then ties the
 // registers of both loads to the wait so that nothing reading them can be
 // scheduled before it.
+// max of three (sm_100's three-input form; NaN handling as fmaxf)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ void regs_after_wait(uint32_t (&r)[32]) {
   asm volatile(
       ""
@@ -401,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
         if (!tail) {
 #pragma unroll
           for (uint32_t e = 0; e < 32; ++e)
-            mx_raw = fmaxf(mx_raw, fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
+            mx_raw = max3f(mx_raw, __uint_as_float(r0[e]), __uint_as_float(r1[e]));
         } else {
 #pragma unroll
           for (uint32_t e = 0; e < 32; ++e) {
@@ -421,7 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
       // pass 2: probabilities 2^(s scale - m), their sum, bf16 into the score
       // buffer's first 64 columns (chunk c's 16 words go over columns already read)
       const float neg_m = -m_run;
-      float sum0 = 0.0f, sum1 = 0.0f;
+      // both halves of a pair of scores on the packed fp32 pipe (the same
+      // roundings as two scalar operations); the sum as fma(p, 1, sum)
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+      const float2 nm2 = make_float2(neg_m, neg_m), one2 = make_float2(1.0f, 1.0f);
+      float2 sum2 = make_float2(0.0f, 0.0f);
 #pragma unroll 1
       for (uint32_t c = 0; c < 4; c += 2) {
         // two 32-column chunks per tensor-memory round trip
@@ -435,22 +446,23 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
 #pragma unroll
           for (uint32_t e = 0; e < 16; ++e) {
             const uint32_t k0 = 32 * (c + h2) + 2 * e;
-            float p0 = exp2_approx(__fmaf_rn(__uint_as_float(r[h2][2 * e]), a.scale_log2, neg_m));
-            float p1 =
-                exp2_approx(__fmaf_rn(__uint_as_float(r[h2][2 * e + 1]), a.scale_log2, neg_m));
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(r[h2][2 * e]), __uint_as_float(r[h2][2 * e + 1])),
+                sc2, nm2);
+            float p0 = exp2_approx(x.x);
+            float p1 = exp2_approx(x.y);
             if (tail) {
               p0 = k0 < n_valid ? p0 : 0.0f;
               p1 = k0 + 1 < n_valid ? p1 : 0.0f;
             }
-            sum0 += p0;
-            sum1 += p1;
+            sum2 = __ffma2_rn(make_float2(p0, p1), one2, sum2);
             pk[e] = bf16x2_rn(p0, p1);
           }
           // P chunk c + h2 -> columns 16 (c + h2): inside chunks already read
           tmem_st16(s_addr + 16 * (c + h2), pk);
         }
       }
-      l_run += sum0 + sum1;
+      l_run += sum2.x + sum2.y;
       // a raised maximum rescales this row's O (tile j-1's P V, complete since
       // S_g of tile j is)
       if (__any_sync(0xFFFFFFFFu, factor != 1.0f) && j > 0) {
