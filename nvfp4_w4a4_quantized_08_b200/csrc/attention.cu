@@ -41,10 +41,11 @@
 //               the L2 latency of those loads hides behind the decoding.
 // Tensor memory (512 columns): O0, O1, S0, S1 at columns 0, 128, 256, 384.
 // The running maximum is raised lazily: while a row's new scores stay within
-// 2^8 of the maximum in use, the probabilities are taken against the old one
-// (they stay <= 2^8); only a larger step rescales the row's O and sum, which
-// is safe at once: S_g of tile j completes after P V of tile j-1 of the same
-// query tile.  Every wait is bounded: one that runs out records
+// 2^16 of the maximum in use, the probabilities are taken against the old one
+// (they stay <= 2^16: bf16 P, the fp32 sum and the fp32 O hold that range with
+// their relative precision unchanged); only a larger step rescales the row's O
+// and sum, which is safe at once: S_g of tile j completes after P V of tile
+// j-1 of the same query tile.  Every wait is bounded: one that runs out records
 // NVFP4_ERR_TIMEOUT in the workspace status word, and the CTA drains its MMAs,
 // frees tensor memory and returns.
 #include "common.cuh"
@@ -87,7 +88,7 @@ constexpr uint32_t kSCol0 = 256;          // S_g (then P_g) at kSCol0 + 128 g
 // 10), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBK >> 3) << 17) |
                             (uint32_t(kBQ >> 4) << 24);
-constexpr float kLazyLog2 = 8.0f;          // largest probability kept before a rescale: 2^8
+constexpr float kLazyLog2 = 16.0f;         // largest probability kept before a rescale: 2^16
 
 struct AttnArgs {
   const uint16_t* q;   // bf16 [tq][q_stride], head h at h * 128
@@ -418,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attention_kernel(const Att
         }
       }
       const float mx = __fmul_rn(mx_raw, a.scale_log2);
-      // lazy maximum: keep the one in use while the tile stays within 2^8 of it
+      // lazy maximum: keep the one in use while the tile stays within 2^16 of it
       float factor = 1.0f;
       if (mx > m_run + kLazyLog2) {
         factor = exp2_approx(m_run - mx);   // 0 on the first tile
