@@ -40,28 +40,26 @@ __device__ __forceinline__ BlockLut make_lut(uint32_t sb, float s_t) {
   return l;
 }
 
-// 8 codes (nibble i of c = element i) -> 8 bf16 in four words.  Magnitudes
-// come from the block table (byte permutes indexed by the 3 magnitude bits);
-// the sign bits are gathered with one more permute per output word: se holds
-// the signs of the even elements at bit 7 of each byte, so those of the odd
-// elements, and the permute places element 2k's byte at byte 1 and element
-// 2k+1's at byte 3 of word k.
+// 8 codes (nibble i of c = element i) -> 8 bf16 in four words.  The low and
+// high bytes of the magnitudes come from the block table (byte permutes
+// indexed by the 3 magnitude bits), then two permutes interleave them into
+// bf16 words.  The sign of element i is bit 4i + 3 of c and belongs at bit 7
+// of its high byte: a permute of (c << 4, c) puts the signs of elements
+// 0, 1, 2, 3 (bits 3, 7, 11, 15 of c) at bit 7 of bytes 0..3, those of
+// elements 4..7 likewise, so one and-or per four high bytes adds them.
 __device__ __forceinline__ uint4 decode8(const BlockLut& l, uint32_t c) {
   const uint32_t m = c & 0x77777777u;
   const uint32_t mh = m >> 16;
+  const uint32_t c4 = c << 4;
   uint4 o;
-  uint32_t lo4 = prmt(l.lo0, l.lo1, m), hi4 = prmt(l.hi0, l.hi1, m);
+  uint32_t lo4 = prmt(l.lo0, l.lo1, m);
+  uint32_t hi4 = prmt(l.hi0, l.hi1, m) | (prmt(c4, c, 0x5140) & 0x80808080u);
   o.x = prmt(lo4, hi4, 0x5140);
   o.y = prmt(lo4, hi4, 0x7362);
   lo4 = prmt(l.lo0, l.lo1, mh);
-  hi4 = prmt(l.hi0, l.hi1, mh);
+  hi4 = prmt(l.hi0, l.hi1, mh) | (prmt(c4, c, 0x7362) & 0x80808080u);
   o.z = prmt(lo4, hi4, 0x5140);
   o.w = prmt(lo4, hi4, 0x7362);
-  const uint32_t se = (c << 4) & 0x80808080u, so = c & 0x80808080u;
-  o.x |= prmt(se, so, 0x4000) & 0x80008000u;
-  o.y |= prmt(se, so, 0x5010) & 0x80008000u;
-  o.z |= prmt(se, so, 0x6020) & 0x80008000u;
-  o.w |= prmt(se, so, 0x7030) & 0x80008000u;
   return o;
 }
 
