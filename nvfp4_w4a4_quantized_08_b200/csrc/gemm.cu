@@ -477,6 +477,7 @@ struct Params {
   uint32_t kslabs;   // ceil(K / 256)
   uint32_t tiles_m, tiles_n;  // output tiles: tiles_m of 128 * kPair rows, tiles_n of 256 cols
   uint32_t sf_row_tiles;      // 128-row blocks of A that exist (ceil(M / 128))
+  uint32_t w_sf_row_tiles;    // 128-row blocks of W that exist (ceil(N / 128))
   uint32_t* status;
   uint32_t* c_amax;  // float bits of max|C| (atomicMax), or null
   uint32_t amax_tiles;  // N tiles per c_amax word (0: one word)
@@ -555,11 +556,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // are loaded
         const uint32_t rt = tm * kPair + rank;
         const bool a_live = rt < p.sf_row_tiles;
+        // the tile's second 128 W rows may lie past the last row block of W
+        // (N not a multiple of 256): their scales are not loaded, and the
+        // output columns they feed are neither stored nor counted in c_amax
+        const uint32_t w_halves = 2 * tn + 1 < p.w_sf_row_tiles ? 2u : 1u;
         for (uint32_t kb = 0; kb < p.kslabs; ++kb) {
           if (!waiter.wait(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
           const uint32_t fb = bar_full + 8 * stage;
-          bar_arrive_expect_tx(fb, kABytes + C::kBBytes + (a_live ? 3u : 2u) * 512u * nk);
+          bar_arrive_expect_tx(fb, kABytes + C::kBBytes + ((a_live ? 1u : 0u) + w_halves) * 512u * nk);
           tma_load_2d(sbase + C::kOffA + stage * kABytes, &map_a, int32_t(kb * kBKBytes),
                       int32_t(rt * kBM), fb);
           tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &map_w, int32_t(kb * kBKBytes),
@@ -568,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_load(sbase + C::kOffSfa + stage * kSfaBytes,
                       p.a_sf + (size_t(rt) * p.ktiles + kb * kKSteps) * 512, 512 * nk, fb);
           // the scales of all 256 W rows of the tile, in either form
-          for (uint32_t h = 0; h < 2; ++h)
+          for (uint32_t h = 0; h < w_halves; ++h)
             bulk_load(sbase + C::kOffSfb + stage * kSfbBytes + h * 2048,
                       p.w_sf + (size_t(2 * tn + h) * p.ktiles + kb * kKSteps) * 512, 512 * nk,
                       fb);
@@ -720,6 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = row0 < p.M;  // warp-uniform: some of the 32 rows exist
       const int32_t y = int32_t(row0);
       const int32_t x0 = int32_t(tn * kBN + half * 128);
+      const int32_t n_left = int32_t(p.N) - x0;  // columns of this warp's 128 that exist
       // warp-uniform outcome: tcgen05.ld below is .sync.aligned
       const bool ok = waiter.wait(bar_acc_full, local & 1);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
@@ -752,14 +758,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 64; ++e) pk[e] = gelu_bf16x2(pk[e]);
         }
         if (row_live) {
+          if (n_left >= 128) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) vmax = __vmaxu2(vmax, pk[e] & 0x7FFF7FFFu);
+            for (int e = 0; e < 64; ++e) vmax = __vmaxu2(vmax, pk[e] & 0x7FFF7FFFu);
+          } else {  // the tile's last columns lie past N
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+              vmax = __vmaxu2(vmax, pk[e] & ((2 * e < n_left ? 0x7FFFu : 0u) |
+                                             (2 * e + 1 < n_left ? 0x7FFF0000u : 0u)));
+          }
         }
         if (store) {
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch)
-            store_row_chunk(*reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * ch]), buf, lane,
-                            &map_c, x0 + 64 * ch, y);
+            if (64 * ch < n_left)  // a chunk past N is not stored (a partial one is clipped)
+              store_row_chunk(*reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * ch]), buf, lane,
+                              &map_c, x0 + 64 * ch, y);
         }
       } else {
 #pragma unroll 1
@@ -772,9 +786,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 3) release();
           if (row_live) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) vmax = max(vmax, v[e] & 0x7FFFFFFFu);
+            for (int e = 0; e < 32; ++e)
+              vmax = max(vmax, 32 * c + e < n_left ? v[e] & 0x7FFFFFFFu : 0u);
           }
-          if (store) store_row_chunk(v, buf, lane, &map_c, x0 + 32 * c, y);
+          if (store && 32 * c < n_left) store_row_chunk(v, buf, lane, &map_c, x0 + 32 * c, y);
         }
       }
     }
@@ -919,7 +934,8 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.ktiles = uint32_t(g.K / 64);
   p.kslabs = uint32_t((g.K + 255) / 256);
   p.tiles_m = uint32_t((g.M + tile_m - 1) / tile_m);
-  p.tiles_n = uint32_t(g.N / gemm::kBN);
+  p.tiles_n = uint32_t((g.N + gemm::kBN - 1) / gemm::kBN);
+  p.w_sf_row_tiles = uint32_t((g.N + gemm::kBM - 1) / gemm::kBM);
   p.sf_row_tiles = uint32_t((g.M + gemm::kBM - 1) / gemm::kBM);
   p.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(g.ws) + kWsStatus);
   p.c_amax = reinterpret_cast<uint32_t*>(g.c_amax);

@@ -96,8 +96,9 @@ def test_gemm_rejects(L):
              *ok_args) == N.ERR_INVALID_ARG  # K mismatch
     assert g(ctypes.byref(_tensor(rows=2640, cols=3056)),
              ctypes.byref(_tensor(rows=9216, cols=3056)), *ok_args) == N.ERR_UNSUPPORTED_SHAPE
+    # any N; a c_amax column group must divide it
     assert g(ctypes.byref(a), ctypes.byref(_tensor(rows=9200, cols=3072)),
-             FAKE, N.BF16, 9216, 0, None, 0, FAKE, 256, None) == N.ERR_UNSUPPORTED_SHAPE  # N % 256
+             FAKE, N.BF16, 9216, 0, FAKE, 3072, FAKE, 256, None) == N.ERR_INVALID_ARG
     assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9000, 0, None, 0, FAKE, 256,
              None) == N.ERR_INVALID_ARG  # ldc < N
     assert g(ctypes.byref(a), ctypes.byref(w), FAKE, N.BF16, 9220, 0, None, 0, FAKE, 256,

@@ -46,7 +46,11 @@ def test_tiny_gemm_all_elements(orc, out_dtype):
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 64), (100, 256, 128), (128, 512, 192),
                                    (129, 256, 320), (300, 768, 1024), (77, 256, 4096),
-                                   (513, 1024, 256)])
+                                   (513, 1024, 256),
+                                   # N tails: a last tile without its second 128 W rows
+                                   # (384, 640), with them partly padding (200), tiny N
+                                   (100, 384, 128), (300, 200, 256), (129, 16, 64),
+                                   (513, 640, 192), (1, 48, 64)])
 def test_small_shapes(orc, M, N, K):
     g = torch.Generator().manual_seed(M * 31 + N * 7 + K)
     a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
@@ -108,7 +112,8 @@ def test_ffn_pair(orc):
 
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (129, 512, 320), (300, 768, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (129, 512, 320), (300, 768, 1024),
+                                   (129, 384, 320)])
 def test_gelu_epilogue(orc, M, N, K, out_dtype):
     """act = GELU (tanh form) in the epilogue, every element against the
     oracle's binary64 GELU of its binary64 GEMM, over inputs that put outputs
@@ -163,3 +168,27 @@ def test_timeout_path_reports_and_recovers(orc):
         assert_gemm_close(y.cpu().numpy(), y_ref, S, False)
     assert all(st in (0, nv._native.ERR_TIMEOUT) for st in seen), seen
     assert nv._native.ERR_TIMEOUT in seen, seen
+
+
+@pytest.mark.parametrize("M,N,K,out_dtype", [(300, 384, 256, torch.bfloat16),
+                                             (129, 200, 128, torch.float32),
+                                             (100, 640, 192, torch.bfloat16)])
+def test_n_tail_amax_and_padding(orc, M, N, K, out_dtype):
+    """A GEMM whose N is not a multiple of the 256-column tile: every stored
+    element within the bound, the c_amax word equal to max|C| over the stored
+    values only (the tile's columns past N hold no output), and the columns of
+    a wider output buffer past N left untouched."""
+    g = torch.Generator().manual_seed(M + 7 * N + 11 * K)
+    a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    qa, qw, oa, ow = _operands(orc, a, w)
+    ldc = (N + 63) // 64 * 64 + 64
+    buf = torch.full((M, ldc), 7.0, dtype=out_dtype, device="cuda")
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    y = nv.gemm(qa, qw, out=buf[:, :N], c_amax=amax)
+    y_ref, S = orc.gemm(oa, ow)
+    assert_gemm_close(y.float().cpu().numpy(), y_ref, S, out_dtype == torch.bfloat16)
+    assert float(amax.cpu()[0]) == float(y.float().abs().max().cpu())
+    assert bool((buf[:, N:] == 7.0).all())
+    assert nv.device_status() == 0
+
