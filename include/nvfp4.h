@@ -203,8 +203,9 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* out, int64
  * (nvfp4_act), then rounded to c_dtype.
  *   A: M x K activations, W: N x K weights (both K-contiguous), both with
  *      sf_layout == NVFP4_SF_MMA128x4 and the same K.
- *   Shapes: K a multiple of 64, M >= 1 and N >= 1 (any M and N; the tiles'
- *      tail rows and columns are masked).
+ *   Shapes: K a multiple of 32, M >= 1 and N >= 1 (any M and N; the tiles'
+ *      tail rows and columns are masked, and a last partial 64-wide K step
+ *      reads zero codes and the scale layout's zero padding).
  *   C: device, c_dtype (bf16 or fp32), row stride ldc >= N elements, ldc a
  *      multiple of 8, 16-byte aligned.
  *   act: nvfp4_act.

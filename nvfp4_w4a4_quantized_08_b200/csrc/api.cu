@@ -173,7 +173,9 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
   if (A->sf_layout != NVFP4_SF_MMA128x4 || W->sf_layout != NVFP4_SF_MMA128x4)
     return NVFP4_ERR_INVALID_ARG;
   if (A->cols != W->cols) return NVFP4_ERR_INVALID_ARG;
-  if (A->cols % 64 != 0 || W->rows < 1) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  // K: whole 16-byte code rows (TMA); a K step past K reads TMA zero fill and the
+  // scale layout's zero padding
+  if (A->cols % 32 != 0 || W->rows < 1) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (A->rows >= (int64_t(1) << 31) || W->rows >= (int64_t(1) << 31))
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (ldc < W->rows) return NVFP4_ERR_INVALID_ARG;

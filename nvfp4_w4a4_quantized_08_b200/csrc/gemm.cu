@@ -473,7 +473,7 @@ struct Params {
   const float* a_st;
   const float* w_st;
   uint32_t M, N;
-  uint32_t ktiles;   // K / 64
+  uint32_t ktiles;   // ceil(K / 64): MMA K steps, scale tiles along K
   uint32_t kslabs;   // ceil(K / 256)
   uint32_t tiles_m, tiles_n;  // output tiles: tiles_m of 128 * kPair rows, tiles_n of 256 cols
   uint32_t sf_row_tiles;      // 128-row blocks of A that exist (ceil(M / 128))
@@ -931,7 +931,7 @@ cudaError_t launch_gemm(const LaunchGemm& g, cudaStream_t st) {
   p.w_st = g.w_st;
   p.M = uint32_t(g.M);
   p.N = uint32_t(g.N);
-  p.ktiles = uint32_t(g.K / 64);
+  p.ktiles = uint32_t((g.K + 63) / 64);  // a last partial K step reads zero codes and scales
   p.kslabs = uint32_t((g.K + 255) / 256);
   p.tiles_m = uint32_t((g.M + tile_m - 1) / tile_m);
   p.tiles_n = uint32_t((g.N + gemm::kBN - 1) / gemm::kBN);

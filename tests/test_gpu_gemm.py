@@ -50,7 +50,10 @@ def test_tiny_gemm_all_elements(orc, out_dtype):
                                    # N tails: a last tile without its second 128 W rows
                                    # (384, 640), with them partly padding (200), tiny N
                                    (100, 384, 128), (300, 200, 256), (129, 16, 64),
-                                   (513, 640, 192), (1, 48, 64)])
+                                   (513, 640, 192), (1, 48, 64),
+                                   # K not a multiple of 64: a last half K step
+                                   (100, 256, 32), (300, 256, 96), (129, 384, 160),
+                                   (1, 200, 288)])
 def test_small_shapes(orc, M, N, K):
     g = torch.Generator().manual_seed(M * 31 + N * 7 + K)
     a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
