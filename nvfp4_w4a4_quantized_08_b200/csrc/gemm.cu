@@ -73,8 +73,10 @@ constexpr int kWriterWarp0 = 2 + kEpiWarps;  // 10
 constexpr int kThreads = (kWriterWarp0 + 4) * 32;  // 448
 constexpr int kTmemCols = 512;
 constexpr int kSfCol = kBN;                  // scale sets after the accumulator
-constexpr int kSfStepCols = 12;              // per K step: SFA at +0, SFB at +4 and +8
-constexpr int kSfSetCols = kKSteps * kSfStepCols;
+// A stage's scale set: the A scales of K step j at columns 4j (lane quadrant q
+// reads column 4j + q), the W scales of K step j at columns 16 + 8j .. 16 + 8j + 7
+constexpr int kSfWCol = 4 * kKSteps;         // 16
+constexpr int kSfSetCols = kSfWCol + 8 * kKSteps;  // 48
 constexpr int kStageBufBytes = 32 * 128;     // epilogue staging: 32 rows x 128 bytes
 
 // Per-form sizes: kPair = 1 (single CTA) or 2 (CTA pair).
@@ -331,17 +333,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// One 32-bit column of this warp's 32 tensor-memory lanes from a register.
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v)
-               : "memory");
+// 16 and 32 consecutive 32-bit columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
 }
-
-// Four consecutive 32-bit columns of this warp's 32 lanes.
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint4 v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
-               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
@@ -610,8 +623,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t b_d = desc_sw128(sbase + C::kOffB + stage * C::kBBytes);
           const uint32_t sf = tmem + kSfCol + kSfSetCols * stage;
           for (uint32_t j = 0; j < nk; ++j)  // K step j: +32 bytes = +2 in the address field
-            tc_mma<kPair>(tmem, a_d + 2 * j, b_d + 2 * j, C::kIdesc, sf + kSfStepCols * j,
-                          sf + kSfStepCols * j + 4, (kb | j) != 0);
+            tc_mma<kPair>(tmem, a_d + 2 * j, b_d + 2 * j, C::kIdesc, sf + 4 * j,
+                          sf + kSfWCol + 8 * j, (kb | j) != 0);
           // frees the shared-memory stage and its scale set (of both CTAs of a
           // pair) once these MMAs complete
           tc_commit<kPair>(bar_empty + 8 * stage);
@@ -652,15 +665,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xFFFFFFFFu, waiter.wait(bar_full + 8 * stage, phase));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t nk = min(uint32_t(kKSteps), p.ktiles - kb * kKSteps);
         const uint32_t sfa_s = sbase + C::kOffSfa + stage * kSfaBytes + 16 * uint32_t(lane) + 4 * q;
         const uint32_t sfb_s = sbase + C::kOffSfb + stage * kSfbBytes + 16 * uint32_t(lane);
         const uint32_t col = tmem + lane_bits + kSfCol + kSfSetCols * stage;
-        for (uint32_t j = 0; j < nk; ++j) {
-          tmem_st1(col + kSfStepCols * j + q, ld_shared_u32(sfa_s + 512 * j));
-          tmem_st4(col + kSfStepCols * j + 4, ld_shared_v4(sfb_s + 512 * j));
-          tmem_st4(col + kSfStepCols * j + 8, ld_shared_v4(sfb_s + 2048 + 512 * j));
+        // the whole set in two stores: A word j repeated over columns 4j..4j+3
+        // (only column 4j + q of these lanes is read), W chunks j over 16 + 8j..
+        // (K steps past nk, in a last partial stage, write values no MMA reads)
+        uint32_t av[16], wv[32];
+#pragma unroll
+        for (int j = 0; j < kKSteps; ++j) {
+          const uint32_t a = ld_shared_u32(sfa_s + 512 * j);
+          const uint4 lo = ld_shared_v4(sfb_s + 512 * j);
+          const uint4 hi = ld_shared_v4(sfb_s + 2048 + 512 * j);
+          av[4 * j] = av[4 * j + 1] = av[4 * j + 2] = av[4 * j + 3] = a;
+          wv[8 * j] = lo.x, wv[8 * j + 1] = lo.y, wv[8 * j + 2] = lo.z, wv[8 * j + 3] = lo.w;
+          wv[8 * j + 4] = hi.x, wv[8 * j + 5] = hi.y, wv[8 * j + 6] = hi.z, wv[8 * j + 7] = hi.w;
         }
+        tmem_st16(col, av);
+        tmem_st32(col + kSfWCol, wv);
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         __syncwarp();
@@ -733,23 +755,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem + ((quad * 32) << 16) + half * 128;
       if (bf16) {
         uint32_t pk[64];
-        // two 32-column loads in flight per wait: the accumulator is released
-        // after two load latencies instead of four
+        auto pack = [&](const uint32_t (&r)[32], int c) {
 #pragma unroll
-        for (int c = 0; c < 4; c += 2) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32_async(taddr + 32 * c, r0);
-          tmem_ld32_async(taddr + 32 * c + 32, r1);
-          tmem_wait_ld2(r0, r1);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            pk[16 * c + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r0[2 * e]), alpha),
-                                       __fmul_rn(__uint_as_float(r0[2 * e + 1]), alpha));
-            pk[16 * c + 16 + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r1[2 * e]), alpha),
-                                            __fmul_rn(__uint_as_float(r1[2 * e + 1]), alpha));
-          }
-        }
+          for (int e = 0; e < 16; ++e)
+            pk[16 * c + e] = bf16x2_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
+                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+        };
+        // two 32-column loads in flight per wait; chunks 2 and 3 are loaded
+        // while chunks 0 and 1 are packed, and the accumulator is released as
+        // soon as the last load has landed, before the last packing
+        uint32_t r0[32], r1[32], r2[32];
+        tmem_ld32_async(taddr, r0);
+        tmem_ld32_async(taddr + 32, r1);
+        tmem_wait_ld2(r0, r1);
+        tmem_ld32_async(taddr + 64, r2);
+        pack(r0, 0);
+        tmem_ld32_async(taddr + 96, r0);
+        pack(r1, 1);
+        tmem_wait_ld2(r2, r0);
         release();
+        pack(r2, 2);
+        pack(r0, 3);
         // the activation runs on the bf16 products once the accumulator is
         // released, overlapping the next tile's MMAs: a bf16 linear layer
         // followed by its activation
