@@ -653,7 +653,7 @@ def run_ours(args):
     ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in_ready", "in_free",
                                                              "out_ready", "out_free")}
 
-    def run_e2e(n):
+    def run_e2e(n, eager=False):
         copy_stream.wait_stream(cur)
         with torch.cuda.stream(copy_stream):
             x_stage[0].copy_(h_in, non_blocking=True)
@@ -670,7 +670,10 @@ def run_ours(args):
             cur.wait_event(ev["in_ready"][b])
             step.x_in.copy_(x_stage[b], non_blocking=True)
             ev["in_free"][b].record(cur)
-            graph.replay()
+            if eager:  # the step's C-ABI calls issued one by one through the binding
+                step.run()
+            else:
+                graph.replay()
             if i >= 2:
                 cur.wait_event(ev["out_free"][b])
             o_stage[b].copy_(step.output(), non_blocking=True)
@@ -694,6 +697,17 @@ def run_ours(args):
     assert torch.equal(h_out[(args.steps - 1) % 2], step.output().cpu())
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     e2e_value = job_throughput(flops_step, world, ms_e2e / args.steps)
+    # the same, with the step's launches issued eagerly every step: the host
+    # side of every C-ABI call (argument checks, tensor maps) in the timed region
+    run_e2e(2, eager=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(cur)
+    run_e2e(args.steps, eager=True)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    assert torch.equal(h_out[(args.steps - 1) % 2], step.output().cpu())
+    ms_e2e_eager = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     status = nv.device_status(step.ws)
     # the KV chunk under Four Over Six (the adaptive KV scale rule; not on the
     # step's path): one layer's 3 new frames of K and V, graph-replayed
@@ -785,7 +799,13 @@ def run_ours(args):
                     "d2h_bytes_per_step": M * D * 2, "ms_per_step": ms_e2e / args.steps,
                     "note": "every step's input from pinned host memory and its result back, "
                             "on a copy stream through two staging buffers each way (overlapping "
-                            "the neighbouring steps' compute), inside the timed region"},
+                            "the neighbouring steps' compute), inside the timed region; the step "
+                            "replays the CUDA graph of its C-ABI calls",
+                    "eager": {"value": job_throughput(flops_step, world, ms_e2e_eager / args.steps),
+                              "ms_per_step": ms_e2e_eager / args.steps,
+                              "note": "the same copies, the step's C-ABI calls issued one by one "
+                                      "through the Python binding every step (their host-side "
+                                      "checks and tensor-map encoding inside the timed region)"}},
             "gpu_launches": step.launches_per_step() * args.steps,
             "clocks": clock_info,
             "device_status": status,
