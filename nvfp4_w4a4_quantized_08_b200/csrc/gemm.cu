@@ -8,10 +8,11 @@
 // accumulated in FP32 in tensor memory; the tensor-scale product s_tA * s_tW
 // is applied once in the epilogue.
 //
-// What sets the speed.  The tensor core finishes a 128 x 256 x 64 FP4 step in
-// about 128 clocks, so it needs each step's operand bytes (and their scales)
-// delivered into the SM that fast; operand delivery from L2, not the tensor
-// pipe, is the limit.  Two things follow:
+// What sets the speed.  The MMAs are issued by one thread, which is held until
+// the tensor pipe accepts each one: a stage of four 256 x 256 x 64 pair MMAs
+// takes ~800 clocks with the scale hand-off, and a 256 x 192 x 64 MMA takes
+// about as long as a 256 x 256 x 64 one, so the tile is as wide as the MMA
+// allows.  The operands and their scales must arrive ahead of that pace:
 //   * bytes per MAC: in the pair form a cluster of two CTAs on two SMs computes
 //     a 256 x 256 tile with one cta_group::2 MMA per K step.  Each CTA stages
 //     its own 128 rows of A and its own half of the tile's 256 W rows, and the
@@ -649,8 +650,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     //   W scales of row n (any of the 256, every quadrant needs them all):
     //     lane 32q + n % 32, column sfb + n / 32.
     // In a pair each CTA's tensor memory holds the same layout for its own 128
-    // rows of A and all 256 W rows of the tile.  So warp q writes word q of A
-    // chunk `lane` into one column and both W chunks `lane` whole (4 columns
+    // rows of A and all 256 W rows of the tile.  So warp q writes A chunk
+    // `lane` (of which word q is read) and both W chunks `lane` whole (4 columns
     // each) into its lanes, a stage at a time, into the stage's scale set, then
     // arrives on the issuing CTA's sf_ready barrier of the stage.  A set is free
     // when its stage is full again: the producer refilled the stage after the
